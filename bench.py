@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the SPECTRE spectral mix on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one pass of the whole path (row pass, slice pass, inverse row pass
+with residual + LayerNorm) over one batch of the bf16 long workload
+(B=1, L=65536, H=8, D=64, F=8192), inputs resident in HBM.  L2 is flushed
+(256 MiB memset) before every timed step; the flush is outside the timed
+interval.  Each step is timed with CUDA events on the launching stream, and
+the three kernels are timed separately through the library's profiled entry
+point.  With N > 1 (torchrun, one process per GPU) every rank mixes its own
+batch -- no data crosses GPUs -- and the reported time is the max over ranks.
+
+The ``e2e`` figure times the host-buffer entry point: per step, H2D copies of
+q, k, v, x, G, gamma, beta from pinned memory, the mix, and the D2H copy of y.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "spectral-mix tokens/s at B1 L65536 H8 D64 bf16; achieved HBM GB/s vs peak"
+WORKLOAD = "bf16_long"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "source": "fallback"}
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def source_hash() -> str:
+    files = sorted(glob.glob(os.path.join(ROOT, "sub_quadratic_attention_b200", "csrc", "*")) +
+                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    h = hashlib.sha1()
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per step from profiles/traffic.txt, if taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None, {}
+    cur = source_hash()
+    per = {}
+    with open(p) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if len(parts) != 4:
+                continue
+            wl, hsh, kern, nbytes = parts
+            if wl == workload and hsh == cur:
+                per[kern] = float(nbytes)
+    if len(per) == 3:
+        return sum(per.values()), per
+    return None, {}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polling thread)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4, "gpu_idle": 0x1,
+        "applications_clocks_setting": 0x2, "sync_boost": 0x10, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, torch_device: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            p = torch.cuda.get_device_properties(torch_device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that, do not guess
+            self.err = repr(e)
+            self.max_mhz = None
+
+    def _loop(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # very short region: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - (t0 + t1) / 2))[:3]
+        mhz = [s[1] for s in inside]
+        mask = 0
+        for s in inside:
+            mask |= s[2]
+        reasons = [k for k, bit in self.REASONS.items() if mask & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def time_oracle_sample(w, inputs, target_s: float):
+    """Time the oracle on the first nch channels (all tokens, all batch rows),
+    growing nch until one call takes about target_s.  Returns
+    (tokens-equivalent per second, seconds, nch, threads)."""
+    import oracle
+
+    nthreads = os.cpu_count() or 1
+    nch = 8
+    while True:
+        t0 = time.perf_counter()
+        oracle.spectre_out(inputs["q"], inputs["k"], inputs["v"], inputs["G"], H=w.H, F=w.F,
+                           c0=0, c1=nch, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or nch >= w.C:
+            break
+        grow = max(2, int(target_s / max(dt, 1e-3)))
+        nch = min(w.C, nch * grow)
+    tokens = w.B * w.L * nch / w.C
+    return tokens / dt, dt, nch, nthreads
+
+
+def reference_arm(args, w, rank, world):
+    if rank != 0:
+        return
+    from sub_quadratic_attention_b200.workloads import make_inputs
+
+    inputs = make_inputs(w)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    # size the sample once, then time every step on that sample
+    rate, dt, nch, nthreads = time_oracle_sample(w, inputs, per_step)
+    import oracle
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.spectre_out(inputs["q"], inputs["k"], inputs["v"], inputs["G"], H=w.H, F=w.F,
+                           c0=0, c1=nch, nthreads=nthreads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    mean = sum(times) / len(times)
+    tokens = w.B * w.L * nch / w.C
+    value = tokens / mean
+    sample = (f"oracle (fp64, own FFT, OpenMP) on channels 0..{nch - 1} of {w.C}, all "
+              f"{w.B * w.L} tokens, pre-LayerNorm output; tokens/s scaled by {nch}/{w.C}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, world):
+    return {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "C": w.C, "F": w.F,
+            "io_dtype": w.dtype, "global_batch": w.B * world, "seq_len": w.L,
+            "parallelism": f"dp{world} (independent batch per rank, no data-path collective)",
+            "l2": "flushed before every timed step (256 MiB memset, outside the timed interval); "
+                  "inputs 268 MB also exceed L2"}
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+def native_arm(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from sub_quadratic_attention_b200 import binding
+    from sub_quadratic_attention_b200.workloads import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inputs = make_inputs(w, seed_offset=rank)
+    d = {k: v.to(dev) for k, v in inputs.items()}
+    y = torch.empty_like(d["x"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps)
+    h = mix.handle
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        binding.spectre_mix_run(h, d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y,
+                                stream)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_host0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        binding.spectre_mix_run_profiled(h, d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"],
+                                         d["beta"], y, events[i], stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    barrier()
+    sampler.stop()
+    clocks = sampler.summary(t_host0, t_host1)
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in events]
+    kern_ms = [[e[j].elapsed_time(e[j + 1]) for e in events] for j in range(3)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = w.B * w.L * world
+    value = tokens_per_step / (ms_per_step * 1e-3)
+
+    # ---- end-to-end through the host-buffer entry point
+    pinned = {k: v.pin_memory() for k, v in inputs.items()}
+    y_host = torch.empty_like(pinned["x"]).pin_memory()
+    for _ in range(2):
+        binding.spectre_mix_run_host(h, pinned["q"], pinned["k"], pinned["v"], pinned["x"],
+                                     pinned["G"], pinned["gamma"], pinned["beta"], y_host, stream)
+    torch.cuda.synchronize()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        binding.spectre_mix_run_host(h, pinned["q"], pinned["k"], pinned["v"], pinned["x"],
+                                     pinned["G"], pinned["gamma"], pinned["beta"], y_host, stream)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_total = sum(e[0].elapsed_time(e[1]) for e in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = tokens_per_step / (e2e_total / args.steps * 1e-3)
+    nelem = w.B * w.L * w.C
+    h2d = 4 * nelem * w.elem_bytes + inputs["G"].numel() * 4 + 2 * w.C * 4
+    d2h = nelem * w.elem_bytes
+
+    # ---- roofline of the path against measured HBM bandwidth
+    peaks = load_peaks()
+    alg_bytes = w.algorithmic_bytes()
+    achieved = alg_bytes / (ms_per_step * 1e-3) / 1e9
+    traffic, per_kernel_traffic = ncu_traffic(w.name)
+    names = ["rows_fwd", "slices", "rows_inv_ln"]
+    kmean = [sum(k) / len(k) for k in kern_ms]
+    ksum = sum(kmean)
+    kernels = [{"name": n, "ms": round(m, 5), "share": round(m / ksum, 4),
+                "dram_bytes": per_kernel_traffic.get(n)} for n, m in zip(names, kmean)]
+    dom = max(range(3), key=lambda i: kmean[i])
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+        "peak_source": f"{peaks['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+        if peaks["source"] == "measured" else "fallback 6.65 TB/s",
+        "scope": "whole path per step (3 launches): algorithmic bytes = q,k,v,x read + "
+                 "G[:, :F] + gamma, beta read + y written",
+        "algorithmic_bytes": alg_bytes, "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
+        "kernels": kernels, "dominant_kernel": names[dom],
+    }
+
+    # ---- CPU baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, nch, nthreads = time_oracle_sample(w, inputs, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"oracle (fp64) on channels 0..{nch - 1} of {w.C}, all {w.B * w.L} "
+                         f"tokens, pre-LayerNorm output, {dt:.1f} s; tokens/s scaled by "
+                         f"{nch}/{w.C}"}
+
+    if world > 1:
+        gathered = [None] * world
+        dist.all_gather_object(gathered, clocks)
+        reasons = sorted({r for c in gathered for r in c.get("reasons", [])})
+        clocks = dict(clocks)
+        clocks["reasons"] = reasons
+        clocks["per_rank_sm_mhz"] = [c.get("sm_mhz") for c in gathered]
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; shapes and distributions of the bf16 long workload)",
+            "config": config_dict(w, world),
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "hbm_gbs_achieved": round(achieved, 2),
+        }
+        print(json.dumps(line), flush=True)
+    mix.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        # launched without torchrun for N > 1, or mismatched: trust the launcher's world size
+        if world == 1 and args.gpus > 1:
+            print(json.dumps({"error": "run N > 1 under torchrun (one process per GPU)"}),
+                  flush=True)
+            sys.exit(2)
+
+    from sub_quadratic_attention_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        native_arm(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

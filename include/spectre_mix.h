@@ -1,0 +1,149 @@
+/*
+ * spectre_mix.h -- C ABI of libspectre_mix, SPECTRE frequency-domain token
+ * mixing on NVIDIA B200 (sm_100a).
+ *
+ * The operation (SPECTRE walk-through, hotelren.com/news/5925787, §2.2
+ * pseudocode, with the §2.3 low-frequency truncation):
+ *
+ *   q, k, v, x, y : [B, L, C] row-major, C = H * D contiguous,
+ *                   channel c = h * D + d belongs to head h.
+ *   for each (b, c):  Q = rfft(q[b,:,c]), K = rfft(k[b,:,c]), V = rfft(v[b,:,c])
+ *                     O_f = Q_f * conj(K_f) * G[h, f] * V_f   for 0 <= f < F
+ *                     O_f = 0                                 for F <= f <= L/2
+ *                     out[b,:,c] = irfft(O, n = L)
+ *   y[b,t,:] = LayerNorm over C of (out[b,t,:] + x[b,t,:]), with gamma, beta, eps
+ *              (biased variance, eps inside the square root).
+ *
+ * The forward transform is unscaled and the inverse is scaled by 1/L.  The
+ * imaginary parts of the DC and Nyquist bins are ignored by the inverse.  The
+ * gate multiplies in as given (any sigmoid is applied by the caller).
+ *
+ * Supported shapes: L = 2^k (8 <= L <= 2^20) or L = 3 * 2^k (12 <= L <= 786432);
+ * 1 <= B <= 65535; H, D >= 1; 1 <= F <= L/2 + 1; R * C * 4 bytes (R = 16, or 64
+ * for L > 2^18) fits one block's shared memory.
+ *
+ * Numbers: q, k, v, x and y are fp32 (SPECTRE_F32) or bf16 (SPECTRE_BF16), all
+ * of one type; G, gamma and beta are always fp32.  Arithmetic is fp32; y in
+ * bf16 is rounded to nearest even.
+ *
+ * Ownership: the caller owns every tensor.  The handle owns its twiddle
+ * tables and its workspace (allocated by spectre_mix_create, freed by
+ * spectre_mix_destroy).
+ *
+ * Errors: every function returns a status code (SPECTRE_OK or a negative
+ * SPECTRE_ERR_*), never throws and never exits.  Device faults of an
+ * asynchronous launch surface at the caller's next synchronisation.
+ */
+#ifndef SPECTRE_MIX_H
+#define SPECTRE_MIX_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct spectre_mix_s *spectre_mix_t;
+
+enum spectre_dtype {
+    SPECTRE_F32 = 0,  /* q, k, v, x, y stored as IEEE fp32 */
+    SPECTRE_BF16 = 1  /* q, k, v, x, y stored as bfloat16 */
+};
+
+enum spectre_status {
+    SPECTRE_OK = 0,
+    SPECTRE_ERR_ARG = -1,           /* a null pointer, a bad size, F, dtype or eps */
+    SPECTRE_ERR_UNSUPPORTED_L = -2, /* L is not 2^k or 3*2^k in the supported range */
+    SPECTRE_ERR_ALIGN = -3,         /* a tensor pointer is not 16-byte aligned */
+    SPECTRE_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
+    SPECTRE_ERR_NOMEM = -5,         /* device or host allocation failed */
+    SPECTRE_ERR_DEVICE = -6         /* no usable sm_100 device, or wrong current device */
+};
+
+/*
+ * Create a plan for one problem shape.  Validates the shape, picks the
+ * decomposition L = R * M, computes the twiddle tables in double precision
+ * on the host (stored as fp32) and allocates the workspace on the current
+ * CUDA device.  Synchronous.
+ *   out   : receives the handle (set to NULL on failure).
+ *   B     : batch rows; L: sequence length; H: heads; D: channels per head.
+ *   F     : number of low-frequency rfft bins kept (F = L/2 + 1 keeps all).
+ *   dtype : SPECTRE_F32 or SPECTRE_BF16.
+ *   eps   : LayerNorm epsilon, > 0.
+ */
+int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F,
+                       int dtype, float eps);
+
+/*
+ * Enqueue one mix on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream).  Asynchronous: returns after the launches are queued.
+ *   q, k, v, x : device, [B, L, C] in the plan's dtype.
+ *   G          : device, fp32 [H, L/2 + 1] (row h is head h's gate).
+ *   gamma, beta: device, fp32 [C].
+ *   y          : device, [B, L, C] in the plan's dtype; may not alias inputs.
+ * Every pointer must be non-null and 16-byte aligned.  One handle must not run
+ * on two streams at once: its workspace is shared by all its runs.
+ */
+int spectre_mix_run(spectre_mix_t h, const void *q, const void *k, const void *v,
+                    const void *x, const float *G, const float *gamma,
+                    const float *beta, void *y, void *stream);
+
+/*
+ * As spectre_mix_run, and also writes the pre-LayerNorm mixer output `out`
+ * as fp32 [B, L, C] to `out_f32` (device, 16-byte aligned) when it is not
+ * NULL.  For verification; the timed path is spectre_mix_run.
+ */
+int spectre_mix_run_debug(spectre_mix_t h, const void *q, const void *k,
+                          const void *v, const void *x, const float *G,
+                          const float *gamma, const float *beta, void *y,
+                          float *out_f32, void *stream);
+
+/*
+ * End-to-end variant taking HOST buffers (same shapes and types as
+ * spectre_mix_run).  Enqueues host-to-device copies of q, k, v, x, G, gamma
+ * and beta into device staging buffers owned by the handle, the mix, and a
+ * device-to-host copy of y, all on `stream`.  The staging buffers are
+ * allocated on the first call (so that call is synchronous and must not be
+ * made during stream capture).  With page-locked host memory the call is
+ * asynchronous: synchronise `stream` before reading y or reusing the inputs.
+ */
+int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k,
+                         const void *v, const void *x, const float *G,
+                         const float *gamma, const float *beta, void *y,
+                         void *stream);
+
+/*
+ * As spectre_mix_run, and also records the CUDA events events[0..3] on
+ * `stream` around the three kernel launches of the path: events[0] before
+ * the row pass, events[1] before the slice pass, events[2] before the
+ * inverse row pass, events[3] after it.  `events` points to 4 cudaEvent_t
+ * created by the caller.  For per-kernel timing; the launches are the same
+ * as spectre_mix_run's.
+ */
+int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k,
+                             const void *v, const void *x, const float *G,
+                             const float *gamma, const float *beta, void *y,
+                             void *const *events, void *stream);
+
+/* Free the handle, its tables, workspace and staging buffers.  NULL-safe.
+ * Synchronises the device the handle lives on before freeing. */
+int spectre_mix_destroy(spectre_mix_t h);
+
+/* Static, human-readable text for a status code. */
+const char *spectre_mix_error_string(int code);
+
+/* Device bytes held by the handle (tables + workspace), 0 for NULL. */
+size_t spectre_mix_workspace_bytes(spectre_mix_t h);
+
+/*
+ * The decomposition the plan chose: L = R * M, with R-point transforms in the
+ * row passes and M-point transforms per frequency slice.  Any out-pointer may
+ * be NULL.  Returns SPECTRE_ERR_ARG for a NULL handle.
+ */
+int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_channel);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECTRE_MIX_H */

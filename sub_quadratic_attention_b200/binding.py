@@ -1,0 +1,209 @@
+"""ctypes binding of libspectre_mix (C ABI in include/spectre_mix.h).
+
+Argument marshalling only: every step of the mix runs in the library's CUDA
+kernels.  The functions carry the C names; :class:`SpectreMix` wraps a handle
+for use with torch tensors.  Importing this module loads the library and
+raises if it has not been built -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspectre_mix.so")
+
+SPECTRE_F32 = 0
+SPECTRE_BF16 = 1
+
+SPECTRE_OK = 0
+SPECTRE_ERR_ARG = -1
+SPECTRE_ERR_UNSUPPORTED_L = -2
+SPECTRE_ERR_ALIGN = -3
+SPECTRE_ERR_CUDA = -4
+SPECTRE_ERR_NOMEM = -5
+SPECTRE_ERR_DEVICE = -6
+
+# every entry point the header declares, with its ctypes signature
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+SIGNATURES = {
+    "spectre_mix_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _i, ctypes.c_float]),
+    "spectre_mix_run": (_i, [_vp] * 10),
+    "spectre_mix_run_debug": (_i, [_vp] * 11),
+    "spectre_mix_run_host": (_i, [_vp] * 10),
+    "spectre_mix_run_profiled": (_i, [_vp] * 11),
+    "spectre_mix_destroy": (_i, [_vp]),
+    "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
+    "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
+    "spectre_mix_plan_info": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+}
+
+
+class SpectreMixError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {spectre_mix_error_string(code)} (status {code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libspectre_mix.so not found at {LIB_PATH}; build it with "
+            "`python -m sub_quadratic_attention_b200.build_lib` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(t) -> Optional[int]:
+    """Device or host address of a tensor, an int address, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libspectre_mix must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(code: int, where: str) -> None:
+    if code != SPECTRE_OK:
+        raise SpectreMixError(code, where)
+
+
+def spectre_mix_error_string(code: int) -> str:
+    return _lib.spectre_mix_error_string(int(code)).decode()
+
+
+def spectre_mix_create(B: int, L: int, H: int, D: int, F: int, dtype: int, eps: float = 1e-5) -> int:
+    h = _vp()
+    _check(_lib.spectre_mix_create(ctypes.byref(h), B, L, H, D, F, dtype, eps), "spectre_mix_create")
+    return h.value
+
+
+def spectre_mix_create_status(B: int, L: int, H: int, D: int, F: int, dtype: int,
+                              eps: float = 1e-5) -> Tuple[int, Optional[int]]:
+    """Raw status and handle (for tests of the error paths)."""
+    h = _vp()
+    code = _lib.spectre_mix_create(ctypes.byref(h), B, L, H, D, F, dtype, eps)
+    return code, h.value
+
+
+def spectre_mix_run(h: int, q, k, v, x, G, gamma, beta, y, stream=None) -> None:
+    _check(_lib.spectre_mix_run(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G), _ptr(gamma),
+                                _ptr(beta), _ptr(y), _stream(stream)), "spectre_mix_run")
+
+
+def spectre_mix_run_status(h: int, q, k, v, x, G, gamma, beta, y, stream=None) -> int:
+    return _lib.spectre_mix_run(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G), _ptr(gamma),
+                                _ptr(beta), _ptr(y), _stream(stream))
+
+
+def spectre_mix_run_debug(h: int, q, k, v, x, G, gamma, beta, y, out_f32, stream=None) -> None:
+    _check(_lib.spectre_mix_run_debug(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G), _ptr(gamma),
+                                      _ptr(beta), _ptr(y), _ptr(out_f32), _stream(stream)),
+           "spectre_mix_run_debug")
+
+
+def spectre_mix_run_host(h: int, q, k, v, x, G, gamma, beta, y, stream=None) -> None:
+    _check(_lib.spectre_mix_run_host(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G), _ptr(gamma),
+                                     _ptr(beta), _ptr(y), _stream(stream)), "spectre_mix_run_host")
+
+
+def spectre_mix_run_profiled(h: int, q, k, v, x, G, gamma, beta, y, events, stream=None) -> None:
+    """``events``: four ``torch.cuda.Event(enable_timing=True)`` recorded around
+    the three kernel launches."""
+    arr = (_vp * 4)(*[e.cuda_event for e in events])
+    _check(_lib.spectre_mix_run_profiled(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G),
+                                         _ptr(gamma), _ptr(beta), _ptr(y),
+                                         ctypes.cast(arr, _vp), _stream(stream)),
+           "spectre_mix_run_profiled")
+
+
+def spectre_mix_destroy(h: Optional[int]) -> None:
+    _check(_lib.spectre_mix_destroy(h), "spectre_mix_destroy")
+
+
+def spectre_mix_workspace_bytes(h: Optional[int]) -> int:
+    return int(_lib.spectre_mix_workspace_bytes(h))
+
+
+def spectre_mix_plan_info(h: int) -> Tuple[int, int, int]:
+    R, M, S = _i(), _i(), _i()
+    _check(_lib.spectre_mix_plan_info(h, ctypes.byref(R), ctypes.byref(M), ctypes.byref(S)),
+           "spectre_mix_plan_info")
+    return R.value, M.value, S.value
+
+
+class SpectreMix:
+    """A plan for one shape, usable with torch CUDA tensors.
+
+    ``mix(q, k, v, x, G, gamma, beta)`` returns y; pass ``out=`` (fp32
+    [B, L, C]) to also receive the pre-LayerNorm mixer output.
+    """
+
+    def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
+                 dtype: str = "bf16", eps: float = 1e-5):
+        self.B, self.L, self.H, self.D = B, L, H, D
+        self.C = H * D
+        self.F = L // 2 + 1 if F is None else F
+        self.dtype_code = SPECTRE_F32 if dtype in ("f32", "float32", "fp32") else SPECTRE_BF16
+        self.eps = eps
+        self.handle = spectre_mix_create(B, L, H, D, self.F, self.dtype_code, eps)
+
+    def __call__(self, q, k, v, x, G, gamma, beta, y=None, out=None, stream=None):
+        import torch
+
+        if y is None:
+            y = torch.empty_like(x)
+        if out is None:
+            spectre_mix_run(self.handle, q, k, v, x, G, gamma, beta, y, stream)
+        else:
+            spectre_mix_run_debug(self.handle, q, k, v, x, G, gamma, beta, y, out, stream)
+        return y
+
+    def run_host(self, q, k, v, x, G, gamma, beta, y, stream=None):
+        spectre_mix_run_host(self.handle, q, k, v, x, G, gamma, beta, y, stream)
+        return y
+
+    @property
+    def workspace_bytes(self) -> int:
+        return spectre_mix_workspace_bytes(self.handle)
+
+    @property
+    def plan(self) -> Tuple[int, int, int]:
+        return spectre_mix_plan_info(self.handle)
+
+    def close(self) -> None:
+        if self.handle is not None:
+            h, self.handle = self.handle, None
+            spectre_mix_destroy(h)
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

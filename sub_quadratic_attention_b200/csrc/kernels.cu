@@ -1,0 +1,556 @@
+// kernels.cu -- the three kernel families of the SPECTRE spectral mixer on
+// sm_100a (SPECTRE walk-through, hotelren.com/news/5925787: §2.2 pseudocode,
+// §2.3 truncation, §3.1 real/imaginary parts carried as separate reals).
+//
+//   spectre_rows_fwd    : q, k, v rows -> R-point real transforms -> A
+//   spectre_slices<M>   : per (b, c, f1) slice: three M-point FFTs, the gated
+//                         product, one inverse M-point FFT -> P
+//   spectre_rows_inv_ln : P -> R-point inverse (real output) -> + x ->
+//                         LayerNorm over C -> y
+//
+// The index algebra is in kernels.cuh.
+#include <cuda_bf16.h>
+
+#include "fft_regs.cuh"
+#include "kernels.cuh"
+
+namespace spectre {
+
+// ---------------------------------------------------------------------------
+// element I/O
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    __device__ __forceinline__ static float load(const float *p) { return __ldg(p); }
+    __device__ __forceinline__ static float2 load2(const float *p) {
+        return __ldg(reinterpret_cast<const float2 *>(p));
+    }
+    __device__ __forceinline__ static void store(float *p, float v) { *p = v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    __device__ __forceinline__ static float load(const __nv_bfloat16 *p) {
+        return __bfloat162float(__ldg(p));
+    }
+    __device__ __forceinline__ static float2 load2(const __nv_bfloat16 *p) {
+        return __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p)));
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// row pass: A[sig][b][c][f1][t2] = w_L^{f1 t2} sum_{t1} w_R^{f1 t1} sig[b][t1 M + t2][c]
+// Block: (CT/2) x TB threads; thread (tx, ty) owns channels 2tx, 2tx+1 of the
+// tile at t2 = tile*TB + ty, packed as one complex signal (c0 + i c1).
+// ---------------------------------------------------------------------------
+template <int R, typename T>
+__global__ void __launch_bounds__(256) spectre_rows_fwd(RowsFwdArgs a) {
+    constexpr int NF = R / 2 + 1;
+    extern __shared__ float4 smem_f4[];
+    float2 *stage = reinterpret_cast<float2 *>(smem_f4);  // [NF][TB][CT + 4]
+    const int CT = a.CT, TB = a.TB, CTP = a.CT + 4;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int b = blockIdx.z;
+    const int t2 = blockIdx.x * TB + ty;
+    const int c0 = blockIdx.y * CT + 2 * tx;
+    const bool live = (t2 < a.M) && (c0 < a.C);
+    const bool has1 = (c0 + 1 < a.C);
+    const size_t rowstride = (size_t)a.M * a.C;
+    const int nthr = blockDim.x * blockDim.y;
+    const int tid = ty * blockDim.x + tx;
+
+#pragma unroll 1
+    for (int sig = 0; sig < 3; sig++) {
+        const T *src = static_cast<const T *>(sig == 0 ? a.q : (sig == 1 ? a.k : a.v));
+        float2 z[R];
+        if (live) {
+            const T *p = src + ((size_t)b * a.L + t2) * a.C + c0;
+            if (a.vec2) {
+#pragma unroll
+                for (int t1 = 0; t1 < R; t1++) z[t1] = Elem<T>::load2(p + t1 * rowstride);
+            } else {
+#pragma unroll
+                for (int t1 = 0; t1 < R; t1++) {
+                    z[t1].x = Elem<T>::load(p + t1 * rowstride);
+                    z[t1].y = has1 ? Elem<T>::load(p + t1 * rowstride + 1) : 0.f;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int t1 = 0; t1 < R; t1++) z[t1] = make_float2(0.f, 0.f);
+        }
+        Dft<R>::run(z);
+        // separate the two real channels, twiddle by w_L^{f1 t2}, stage
+#pragma unroll
+        for (int f1 = 0; f1 < NF; f1++) {
+            float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
+            float2 xa = cscale(cadd(zf, zc), 0.5f);
+            float2 d = csub(zf, zc);
+            float2 xb = make_float2(0.5f * d.y, -0.5f * d.x);
+            if (f1 > 0 && live) {
+                float2 w = __ldg(a.twL + f1 * t2);
+                xa = cmul(xa, w);
+                xb = cmul(xb, w);
+            }
+            *reinterpret_cast<float4 *>(stage + (f1 * TB + ty) * CTP + 2 * tx) =
+                make_float4(xa.x, xa.y, xb.x, xb.y);
+        }
+        __syncthreads();
+        // store segments of TB consecutive t2 per (c, f1)
+        const int total = CT * NF * TB;
+        float2 *dst = a.A + (size_t)(sig * a.B + b) * a.C * NF * a.M;
+        for (int i = tid; i < total; i += nthr) {
+            int tl = i % TB, rest = i / TB;
+            int cl = rest % CT, f1 = rest / CT;
+            int c = blockIdx.y * CT + cl, tt = blockIdx.x * TB + tl;
+            if (c < a.C && tt < a.M)
+                dst[((size_t)c * NF + f1) * a.M + tt] = stage[(f1 * TB + tl) * CTP + cl];
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// slice pass
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int spad(int i) { return i + (i >> 4); }
+
+// One in-place Stockham pass over shared memory:
+//   butterfly bf < M/R reads buf[bf + r M/R], twiddles by w_{Ns R}^{(bf mod Ns) r},
+//   and writes buf[(bf / Ns) Ns R + (bf mod Ns) + r Ns].
+template <int R, int M, int NT, int NS>
+__device__ __forceinline__ void smem_pass(float2 *buf, const float2 *__restrict__ tw, int j) {
+    constexpr int NBF = M / R;
+    constexpr int NB = (NBF + NT - 1) / NT;
+    float2 v[NB][R];
+#pragma unroll
+    for (int i = 0; i < NB; i++) {
+        int bf = j + i * NT;
+        if (NBF % NT == 0 || bf < NBF) {
+#pragma unroll
+            for (int r = 0; r < R; r++) v[i][r] = buf[spad(bf + r * NBF)];
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < NB; i++) {
+        int bf = j + i * NT;
+        if (NBF % NT == 0 || bf < NBF) {
+            int kk = bf % NS;
+            if (NS > 1) {
+                const float2 *t = tw + kk * R;
+#pragma unroll
+                for (int r = 1; r < R; r++) v[i][r] = cmul(v[i][r], __ldg(t + r));
+            }
+            Dft<R>::run(v[i]);
+            int idxD = (bf / NS) * NS * R + kk;
+#pragma unroll
+            for (int r = 0; r < R; r++) buf[spad(idxD + r * NS)] = v[i][r];
+        }
+    }
+    __syncthreads();
+}
+
+template <int M, int NT, int D, int P, int PEND> struct MidPasses {
+    __device__ __forceinline__ static void run(float2 *buf, const SliceTables &tb, int j) {
+        if constexpr (P < PEND) {
+            constexpr int R = sched_radix(M, D, P);
+            constexpr int NS = sched_stride(M, D, P);
+            smem_pass<R, M, NT, NS>(buf, tb.tw[D][P], j);
+            MidPasses<M, NT, D, P + 1, PEND>::run(buf, tb, j);
+        }
+    }
+};
+
+template <int M> struct SliceCfg {
+    static constexpr RadList S = make_schedule(M);
+    static constexpr int NP = S.n;
+    static constexpr int RL = NP > 0 ? S.r[NP - 1] : 1;   // largest radix, last
+    static constexpr int R0 = NP > 0 ? S.r[0] : 1;
+    static constexpr int NT = M / RL;                      // threads per slice
+    static constexpr int SPB = NT >= 256 ? 1 : 256 / NT;   // slices per block
+    static constexpr int THREADS = NT * SPB;
+    static constexpr int BUF = NP >= 2 ? (M + M / 16) : 0; // float2 per slice
+    static constexpr bool S_IN_REGS = NT <= 512;
+};
+
+// Forward M-point transform of one slice of A.  On return thread j holds
+// X[j + r NT], r < RL, in x[].  buf must not be in use by other threads'
+// loads (callers separate uses with a barrier).
+template <int M>
+__device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bool live, float2 *buf,
+                                              const SliceTables &tb, int j, float2 (&x)[SliceCfg<M>::RL]) {
+    using Cfg = SliceCfg<M>;
+    constexpr int NP = Cfg::NP, NT = Cfg::NT;
+    if constexpr (NP == 0) {
+        x[0] = live ? __ldg(src) : make_float2(0.f, 0.f);
+    } else if constexpr (NP == 1) {
+        constexpr int R = Cfg::RL;
+#pragma unroll
+        for (int r = 0; r < R; r++) x[r] = live ? __ldg(src + j + r * NT) : make_float2(0.f, 0.f);
+        Dft<R>::run(x);
+    } else {
+        // first pass: global -> registers -> smem (Ns = 1, no twiddle)
+        constexpr int R = Cfg::R0;
+        constexpr int NBF = M / R;
+        constexpr int NB = (NBF + NT - 1) / NT;
+#pragma unroll
+        for (int i = 0; i < NB; i++) {
+            int bf = j + i * NT;
+            if (NBF % NT == 0 || bf < NBF) {
+                float2 v[R];
+#pragma unroll
+                for (int r = 0; r < R; r++) v[r] = live ? __ldg(src + bf + r * NBF) : make_float2(0.f, 0.f);
+                Dft<R>::run(v);
+#pragma unroll
+                for (int r = 0; r < R; r++) buf[spad(bf * R + r)] = v[r];
+            }
+        }
+        __syncthreads();
+        MidPasses<M, NT, 0, 1, NP - 1>::run(buf, tb, j);
+        // last pass: smem -> registers, one butterfly per thread (Ns = NT)
+        constexpr int RL = Cfg::RL;
+#pragma unroll
+        for (int r = 0; r < RL; r++) x[r] = buf[spad(j + r * NT)];
+        const float2 *t = tb.tw[0][NP - 1] + j * RL;
+#pragma unroll
+        for (int r = 1; r < RL; r++) x[r] = cmul(x[r], __ldg(t + r));
+        Dft<RL>::run(x);
+    }
+}
+
+// Inverse (unscaled) M-point transform of the values thread j holds at
+// positions j + r NT, via conj -> forward passes in reversed radix order ->
+// conj; writes P[t2] = w_L^{-f1 t2} * result[t2].
+template <int M>
+__device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL], float2 *buf,
+                                                    const SliceTables &tb, int j, bool live,
+                                                    float2 *__restrict__ dst, const float2 *__restrict__ twL,
+                                                    int f1) {
+    using Cfg = SliceCfg<M>;
+    constexpr int NP = Cfg::NP, NT = Cfg::NT, RL = Cfg::RL;
+#pragma unroll
+    for (int r = 0; r < RL; r++) o[r] = cconj(o[r]);
+    if constexpr (NP == 0) {
+        if (live) dst[0] = cconj(o[0]);  // f1 * 0 = 0: no twiddle
+    } else if constexpr (NP == 1) {
+        Dft<RL>::run(o);
+        // single butterfly (j = 0): output r at position r
+        if (live) {
+#pragma unroll
+            for (int r = 0; r < RL; r++) {
+                float2 w = __ldg(twL + f1 * r);
+                dst[r] = cconj(cmul(o[r], w));
+            }
+        }
+    } else {
+        // first inverse pass: radix RL, Ns = 1, registers -> smem
+        Dft<RL>::run(o);
+        __syncthreads();  // the forward's last-pass loads are done everywhere
+#pragma unroll
+        for (int r = 0; r < RL; r++) buf[spad(j * RL + r)] = o[r];
+        __syncthreads();
+        MidPasses<M, NT, 1, 1, NP - 1>::run(buf, tb, j);
+        // last inverse pass: radix R0, Ns = M / R0
+        constexpr int R = Cfg::R0;
+        constexpr int NBF = M / R;
+        constexpr int NB = (NBF + NT - 1) / NT;
+        const float2 *tw = tb.tw[1][NP - 1];
+#pragma unroll
+        for (int i = 0; i < NB; i++) {
+            int bf = j + i * NT;
+            if (NBF % NT == 0 || bf < NBF) {
+                float2 v[R];
+#pragma unroll
+                for (int r = 0; r < R; r++) v[r] = buf[spad(bf + r * NBF)];
+#pragma unroll
+                for (int r = 1; r < R; r++) v[r] = cmul(v[r], __ldg(tw + bf * R + r));
+                Dft<R>::run(v);
+                if (live) {
+#pragma unroll
+                    for (int r = 0; r < R; r++) {
+                        int t2 = bf + r * NBF;
+                        float2 w = __ldg(twL + f1 * t2);
+                        dst[t2] = cconj(cmul(v[r], w));
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int M>
+__global__ void __launch_bounds__(SliceCfg<M>::THREADS) spectre_slices(SliceArgs a) {
+    using Cfg = SliceCfg<M>;
+    constexpr int NT = Cfg::NT, RL = Cfg::RL;
+    extern __shared__ float4 smem_f4[];
+    const int sl = threadIdx.x / NT;
+    const int j = threadIdx.x % NT;
+    float2 *buf = reinterpret_cast<float2 *>(smem_f4) + sl * Cfg::BUF;
+    const long long sid = (long long)blockIdx.x * Cfg::SPB + sl;
+    const bool live = sid < a.nslices;
+    const int NF = a.R / 2 + 1;
+    const long long sidc = live ? sid : 0;
+    const int f1 = (int)(sidc % NF);
+    const long long bc = sidc / NF;             // b * C + c
+    const int c = (int)(bc % a.C);
+    const int h = c / a.D;
+    const size_t sig_stride = (size_t)a.B * a.C * NF * M;
+    const float2 *srcA = a.A + (size_t)bc * NF * M + (size_t)f1 * M;
+    float2 *dstP = a.P + (size_t)bc * NF * M + (size_t)f1 * M;
+    const float *Gh = a.G + (size_t)h * a.nbins;
+
+    float2 x[RL];
+    float2 s[RL];
+    // q: S = Q * G' / L on this thread's bins f = f1 + R (j + r NT)
+    slice_forward<M>(srcA, live, buf, a.tabs, j, x);
+#pragma unroll
+    for (int r = 0; r < RL; r++) {
+        int f = f1 + a.R * (j + r * NT);
+        int ff = min(f, a.L - f);
+        float g = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
+        s[r] = cscale(x[r], g);
+    }
+    if constexpr (!Cfg::S_IN_REGS) {
+        // park S in this slice's P row (rewritten at the end)
+        if (live) {
+#pragma unroll
+            for (int r = 0; r < RL; r++) dstP[j + r * NT] = s[r];
+        }
+    }
+    if constexpr (Cfg::NP >= 2) __syncthreads();
+    // k: S *= conj(K)
+    slice_forward<M>(srcA + sig_stride, live, buf, a.tabs, j, x);
+    if constexpr (!Cfg::S_IN_REGS) {
+#pragma unroll
+        for (int r = 0; r < RL; r++) s[r] = live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < RL; r++) s[r] = cmulc(s[r], x[r]);
+    if constexpr (!Cfg::S_IN_REGS) {
+        if (live) {
+#pragma unroll
+            for (int r = 0; r < RL; r++) dstP[j + r * NT] = s[r];
+        }
+    }
+    if constexpr (Cfg::NP >= 2) __syncthreads();
+    // v: O = S * V
+    slice_forward<M>(srcA + 2 * sig_stride, live, buf, a.tabs, j, x);
+    if constexpr (!Cfg::S_IN_REGS) {
+#pragma unroll
+        for (int r = 0; r < RL; r++) s[r] = live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < RL; r++) x[r] = cmul(s[r], x[r]);
+    slice_inverse_store<M>(x, buf, a.tabs, j, live, dstP, a.twL, f1);
+}
+
+// ---------------------------------------------------------------------------
+// inverse row pass + residual + LayerNorm
+// ---------------------------------------------------------------------------
+template <int R, typename T, bool DEBUG_OUT>
+__global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
+    constexpr int NF = R / 2 + 1;
+    extern __shared__ float4 smem_f4[];
+    float *zbuf = reinterpret_cast<float *>(smem_f4);  // [R * T2C][ZS]
+    const int T2C = a.T2C, ZS = a.ZS;
+    const int b = blockIdx.y;
+    const int t2base = blockIdx.x * T2C;
+    const int CP = (a.C + 1) / 2;
+    const int items = T2C * CP;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int tl = it % T2C, cp = it / T2C;
+        const int t2 = t2base + tl;
+        if (t2 >= a.M) continue;
+        const int c0 = 2 * cp;
+        const bool has1 = c0 + 1 < a.C;
+        const float2 *pa = a.P + ((size_t)b * a.C + c0) * NF * a.M + t2;
+        const float2 *pb = pa + (size_t)NF * a.M;
+        float2 Z[R];
+        {
+            float2 a0 = __ldg(pa), aN = __ldg(pa + (size_t)(R / 2) * a.M);
+            float2 b0 = has1 ? __ldg(pb) : make_float2(0.f, 0.f);
+            float2 bN = has1 ? __ldg(pb + (size_t)(R / 2) * a.M) : make_float2(0.f, 0.f);
+            // DC and Nyquist: imaginary parts dropped; conj() for the inverse
+            Z[0] = make_float2(a0.x, -b0.x);
+            Z[R / 2] = make_float2(aN.x, -bN.x);
+        }
+#pragma unroll
+        for (int f1 = 1; f1 < R / 2; f1++) {
+            float2 pv = __ldg(pa + (size_t)f1 * a.M);
+            float2 qv = has1 ? __ldg(pb + (size_t)f1 * a.M) : make_float2(0.f, 0.f);
+            // Z[f1] = P_a + i P_b ; Z[R - f1] = conj(P_a) + i conj(P_b); stored conjugated
+            Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
+            Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
+        }
+        Dft<R>::run(Z);
+        // inverse result = conj(Z): real part -> channel c0, imaginary -> c0 + 1
+        float *zr = zbuf + (size_t)tl * ZS + c0;
+#pragma unroll
+        for (int t1 = 0; t1 < R; t1++) {
+            float *p = zr + (size_t)t1 * T2C * ZS;
+            if (has1)
+                *reinterpret_cast<float2 *>(p) = make_float2(Z[t1].x, -Z[t1].y);
+            else
+                p[0] = Z[t1].x;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    const T *x = static_cast<const T *>(a.x);
+    T *y = static_cast<T *>(a.y);
+    const float invC = 1.0f / (float)a.C;
+    for (int row = warp; row < R * T2C; row += nw) {
+        const int t1 = row / T2C, tl = row % T2C;
+        const int t2 = t2base + tl;
+        if (t2 >= a.M) continue;
+        const size_t tok = (size_t)b * a.L + (size_t)t1 * a.M + t2;
+        const T *xr = x + tok * a.C;
+        T *yr = y + tok * a.C;
+        float *zr = zbuf + (size_t)row * ZS;
+        float s = 0.f;
+        for (int c = lane; c < a.C; c += 32) {
+            float o = zr[c];
+            if (DEBUG_OUT) a.out_f32[tok * a.C + c] = o;
+            float z = o + Elem<T>::load(xr + c);
+            zr[c] = z;
+            s += z;
+        }
+        const float mean = warp_sum(s) * invC;
+        float ss = 0.f;
+        for (int c = lane; c < a.C; c += 32) {
+            float d = zr[c] - mean;
+            ss = fmaf(d, d, ss);
+        }
+        const float rstd = rsqrtf(warp_sum(ss) * invC + a.eps);
+        for (int c = lane; c < a.C; c += 32)
+            Elem<T>::store(yr + c, fmaf((zr[c] - mean) * rstd, __ldg(a.gamma + c), __ldg(a.beta + c)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+template <int R>
+static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a, cudaStream_t s) {
+    constexpr int NF = R / 2 + 1;
+    dim3 block(a.CT / 2, a.TB);
+    dim3 grid((a.M + a.TB - 1) / a.TB, (a.C + a.CT - 1) / a.CT, a.B);
+    size_t smem = (size_t)NF * a.TB * (a.CT + 4) * sizeof(float2);
+    if (dtype == 0) {
+        auto k = spectre_rows_fwd<R, float>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, block, smem, s>>>(a);
+    } else {
+        auto k = spectre_rows_fwd<R, __nv_bfloat16>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, block, smem, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rows_fwd(int R, int dtype, const RowsFwdArgs &a, cudaStream_t s) {
+    switch (R) {
+    case 4: return rows_fwd_R<4>(dtype, a, s);
+    case 8: return rows_fwd_R<8>(dtype, a, s);
+    case 16: return rows_fwd_R<16>(dtype, a, s);
+    case 64: return rows_fwd_R<64>(dtype, a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int M>
+static cudaError_t slices_M(const SliceArgs &a, cudaStream_t s) {
+    using Cfg = SliceCfg<M>;
+    size_t smem = (size_t)Cfg::BUF * Cfg::SPB * sizeof(float2);
+    long long nblk = (a.nslices + Cfg::SPB - 1) / Cfg::SPB;
+    auto k = spectre_slices<M>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<(unsigned)nblk, Cfg::THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int M> static void slice_geom_M(int *nt, int *spb, size_t *smem) {
+    using Cfg = SliceCfg<M>;
+    *nt = Cfg::NT;
+    *spb = Cfg::SPB;
+    *smem = (size_t)Cfg::BUF * Cfg::SPB * sizeof(float2);
+}
+
+#define SPECTRE_SLICE_LENGTHS(X)                                                              \
+    X(1) X(2) X(4) X(8) X(16) X(32) X(64) X(128) X(256) X(512) X(1024) X(2048) X(4096)     \
+    X(8192) X(16384) X(3) X(6) X(12) X(24) X(48) X(96) X(192) X(384) X(768) X(1536) X(3072) \
+    X(6144) X(12288)
+
+cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s) {
+    switch (a.M) {
+#define X(m) case m: return slices_M<m>(a, s);
+        SPECTRE_SLICE_LENGTHS(X)
+#undef X
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+bool slice_length_supported(int M) {
+    switch (M) {
+#define X(m) case m: return true;
+        SPECTRE_SLICE_LENGTHS(X)
+#undef X
+    default: return false;
+    }
+}
+
+void slice_geometry(int M, int *nt, int *spb, size_t *smem) {
+    *nt = 0;
+    *spb = 0;
+    *smem = 0;
+    switch (M) {
+#define X(m) case m: slice_geom_M<m>(nt, spb, smem); break;
+        SPECTRE_SLICE_LENGTHS(X)
+#undef X
+    default: break;
+    }
+}
+
+template <int R, typename T>
+static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
+    dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
+    size_t smem = (size_t)R * a.T2C * a.ZS * sizeof(float);
+    if (a.out_f32) {
+        auto k = spectre_rows_inv_ln<R, T, true>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, 512, smem, s>>>(a);
+    } else {
+        auto k = spectre_rows_inv_ln<R, T, false>;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k<<<grid, 512, smem, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <int R>
+static cudaError_t rows_inv_R(int dtype, const RowsInvArgs &a, cudaStream_t s) {
+    return dtype == 0 ? rows_inv_RT<R, float>(a, s) : rows_inv_RT<R, __nv_bfloat16>(a, s);
+}
+
+cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStream_t s) {
+    switch (R) {
+    case 4: return rows_inv_R<4>(dtype, a, s);
+    case 8: return rows_inv_R<8>(dtype, a, s);
+    case 16: return rows_inv_R<16>(dtype, a, s);
+    case 64: return rows_inv_R<64>(dtype, a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t upload_w64(const float2 *host64) {
+    return cudaMemcpyToSymbol(c_w64, host64, 64 * sizeof(float2));
+}
+
+}  // namespace spectre

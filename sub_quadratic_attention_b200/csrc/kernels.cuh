@@ -1,0 +1,119 @@
+// kernels.cuh -- launch interface between the plan (api.cu) and the three
+// kernel families of the SPECTRE mixer (rows_fwd.cu, slices.cu, rows_inv_ln.cu).
+//
+// Decomposition (four-step Cooley-Tukey along L, split L = R * M, token
+// t = t1 * M + t2, rfft bin f = f1 + R * f2):
+//   row pass      A[f1][t2] = w_L^{f1 t2} * sum_{t1<R} w_R^{f1 t1} x[t1 M + t2]
+//                 (f1 in [0, R/2]: the real-input half; pairs of channels
+//                 share one complex R-point transform)
+//   slice pass    X[f1 + R f2] = DFT_M(A[f1][.])[f2] for q, k, v; the gated
+//                 product O = Q conj(K) G' V / L on those bins (G' mirrors G
+//                 to f > L/2 and is 0 where min(f, L-f) >= F); then
+//                 P[f1][t2] = w_L^{-f1 t2} * IDFT_M(O[f1 + R .])[t2]
+//   inverse rows  out[t1 M + t2] = sum_{f1<R} w_R^{-f1 t1} P~[f1][t2], with P~
+//                 the Hermitian extension P~[R - f1] = conj(P[f1]); then
+//                 residual + LayerNorm over C on whole token rows.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace spectre {
+
+constexpr int kMaxPasses = 6;
+
+// Per-pass twiddle tables of the M-point slice transforms.  Pass p of
+// direction d (0 = forward radix order, 1 = reversed) with radix R_p and
+// stride Ns_p (product of the earlier radices) uses
+//   tw[d][p][k * R_p + r] = exp(-2 pi i k r / (Ns_p R_p)),  k < Ns_p, r < R_p.
+struct SliceTables {
+    const float2 *tw[2][kMaxPasses];
+};
+
+struct RowsFwdArgs {
+    const void *q, *k, *v;
+    float2 *A;            // [3][B][C][R/2+1][M]
+    const float2 *twL;    // exp(-2 pi i e / L), e in [0, L/2]
+    int B, L, M, C;
+    int CT, TB;           // channel tile, t2 tile
+    int vec2;             // C even: load channel pairs as one vector
+};
+
+struct SliceArgs {
+    const float2 *A;      // [3][B][C][R/2+1][M]
+    float2 *P;            // [B][C][R/2+1][M]
+    const float2 *twL;
+    const float *G;       // [H][L/2+1]
+    SliceTables tabs;
+    int B, L, R, M, C, D, F, nbins;
+    long long nslices;    // B * C * (R/2+1)
+    float invL;
+};
+
+struct RowsInvArgs {
+    const float2 *P;
+    const void *x;
+    const float *gamma, *beta;
+    void *y;
+    float *out_f32;       // nullable
+    int B, L, M, C;
+    int T2C, ZS;          // t2 values per block, padded row stride of the z buffer
+    float eps;
+};
+
+// Returns cudaSuccess or the launch error.  dtype: 0 fp32, 1 bf16.
+cudaError_t launch_rows_fwd(int R, int dtype, const RowsFwdArgs &a, cudaStream_t s);
+cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s);
+cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStream_t s);
+
+// Slice-transform schedule for length M (radices ascending, largest last).
+struct RadList {
+    int n;
+    int r[kMaxPasses];
+};
+
+constexpr RadList make_schedule(int M) {
+    RadList s{0, {0, 0, 0, 0, 0, 0}};
+    int m = M;
+    bool three = false;
+    if (m % 3 == 0) {
+        three = true;
+        m /= 3;
+    }
+    int k = 0;
+    while ((1 << k) < m) k++;
+    int n16 = k / 4, rem = 1 << (k % 4);
+    if (rem > 1) s.r[s.n++] = rem;
+    if (three) s.r[s.n++] = 3;
+    for (int i = 0; i < n16; i++) s.r[s.n++] = 16;
+    for (int i = 0; i < s.n; i++)
+        for (int j = 0; j + 1 < s.n - i; j++)
+            if (s.r[j] > s.r[j + 1]) {
+                int t = s.r[j];
+                s.r[j] = s.r[j + 1];
+                s.r[j + 1] = t;
+            }
+    return s;
+}
+
+// Radix and stride of pass p in direction d (0 forward order, 1 reversed).
+constexpr int sched_radix(int M, int d, int p) {
+    RadList s = make_schedule(M);
+    return d == 0 ? s.r[p] : s.r[s.n - 1 - p];
+}
+constexpr int sched_stride(int M, int d, int p) {
+    int ns = 1;
+    for (int i = 0; i < p; i++) ns *= sched_radix(M, d, i);
+    return ns;
+}
+
+// whether M is a supported slice length (2^k <= 16384 or 3*2^k <= 12288)
+bool slice_length_supported(int M);
+// threads per slice and slices per block the slice kernel uses for M
+void slice_geometry(int M, int *threads_per_slice, int *slices_per_block, size_t *smem_bytes);
+
+// Upload exp(-2 pi i e / 64), e < 64, to the constant bank of the current device.
+cudaError_t upload_w64(const float2 *host64);
+
+}  // namespace spectre

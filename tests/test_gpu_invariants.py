@@ -1,0 +1,76 @@
+"""Properties of the CUDA path that hold at any size, checked at the full
+workload sizes without the oracle (SPECTRE walk-through §2.2: the implied
+L x L mixing matrix is circulant; §2.3: truncation keeps bins f < F).
+
+* a common circular shift of q and k leaves out unchanged;
+* a circular shift of v shifts out by the same amount;
+* out is linear in each of q, k, v (exactly, for a power-of-two scale);
+* q = k = v = cos(2 pi a t / L) gives out = (L^2 / 4) G[a] cos(2 pi a t / L)
+  when a < F and 0 otherwise.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import rel_l2
+from sub_quadratic_attention_b200.workloads import WORKLOADS, custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _out(w, d):
+    from sub_quadratic_attention_b200.binding import SpectreMix
+
+    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps) as mix:
+        y = torch.empty_like(d["x"])
+        out = torch.empty((w.B, w.L, w.C), dtype=torch.float32, device="cuda")
+        mix(d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y=y, out=out)
+        torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("name", ["bf16_long", "bf16_mixed_radix", "bf16_very_long"])
+def test_shift_and_scale_invariants(name):
+    w = WORKLOADS[name]
+    d = {k: v.cuda() for k, v in make_inputs(w).items()}
+    base = _out(w, d)
+    s = w.L // 3 + 7
+    e = dict(d)
+    e["q"] = torch.roll(d["q"], s, 1)
+    e["k"] = torch.roll(d["k"], s, 1)
+    same = _out(w, e)
+    assert rel_l2(same.cpu().numpy(), base.double().cpu().numpy()) < 2e-5
+    e = dict(d)
+    e["v"] = torch.roll(d["v"], s, 1)
+    shifted = _out(w, e)
+    assert rel_l2(shifted.cpu().numpy(), torch.roll(base, s, 1).double().cpu().numpy()) < 2e-5
+    for key in ("q", "k", "v"):
+        e = dict(d)
+        e[key] = d[key] * 2
+        assert torch.equal(_out(w, e), base * 2), key
+
+
+@pytest.mark.parametrize("L,F", [(65536, 8192), (1048576, 65536), (12288, 6145)])
+def test_single_tone_closed_form(L, F):
+    w = custom(1, L, 2, 1, F, dtype="f32")
+    t = torch.arange(L, dtype=torch.float64)
+    g = torch.Generator().manual_seed(L)
+    G = torch.rand(w.H, L // 2 + 1, generator=g, dtype=torch.float32)
+    for a in (1, F - 1, F, L // 2 - 1):
+        if a >= L // 2:
+            continue
+        col = torch.cos(2 * math.pi * a * t / L).to(torch.float32)
+        q = col.reshape(1, L, 1).expand(1, L, w.C).contiguous()
+        d = {"q": q.cuda(), "k": q.cuda(), "v": q.cuda(), "x": torch.zeros_like(q).cuda(),
+             "G": G.cuda(), "gamma": torch.ones(w.C).cuda(), "beta": torch.zeros(w.C).cuda()}
+        out = _out(w, d).cpu().double()
+        scale = L * L / 4
+        for c in range(w.C):
+            if a < F:
+                expect = scale * float(G[c // w.D, a]) * col.double()
+                err = float((out[0, :, c] - expect).abs().max()) / scale
+            else:
+                err = float(out[0, :, c].abs().max()) / scale
+            assert err < 2e-5, (a, c, err)

@@ -1,0 +1,114 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Element-by-element comparisons on the same seeded inputs: every workload at its
+full size (in the launch configuration the benchmark times), a sweep of small
+shapes spanning several tiles with ragged tails, and the degenerate cases of the
+method (F = 1, zero gate, no truncation, odd channel counts, one token block).
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import TOL, check_parity, oracle_full, run_library
+from sub_quadratic_attention_b200.workloads import WORKLOADS, custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "fp32_mid", "bf16_long", "bf16_mixed_radix",
+                                  "bf16_very_long"])
+def test_workload_full_size(name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    out, y = run_library(w, inp)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"{name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+SWEEP = [
+    # (B, L, H, D, F)
+    (1, 8, 1, 2, 5), (2, 12, 1, 3, 7), (1, 16, 2, 2, 9), (3, 24, 1, 5, 4), (1, 32, 1, 4, 17),
+    (1, 48, 3, 5, 25), (2, 64, 2, 3, 1), (1, 96, 1, 7, 30), (1, 128, 4, 4, 65), (2, 192, 2, 8, 50),
+    (1, 256, 1, 16, 129), (1, 384, 3, 3, 100), (1, 512, 2, 32, 257), (1, 768, 1, 24, 385),
+    (2, 1024, 2, 16, 200), (1, 1536, 3, 10, 769), (1, 2048, 1, 64, 1025), (1, 3072, 2, 6, 1000),
+    (1, 4096, 4, 16, 2049), (1, 6144, 1, 40, 3073), (1, 8192, 2, 8, 1024), (1, 12288, 1, 66, 6145),
+    (1, 16384, 1, 32, 8193), (1, 32768, 1, 16, 4000), (1, 65536, 1, 8, 32769),
+    (1, 3 * 2 ** 16, 1, 4, 1234), (1, 2 ** 18, 1, 4, 2 ** 17 + 1), (1, 2 ** 19, 1, 2, 5000),
+    (1, 3 * 2 ** 17, 1, 2, 3 * 2 ** 16 + 1),
+]
+
+
+@pytest.mark.parametrize("B,L,H,D,F", SWEEP)
+def test_shape_sweep_fp32(B, L, H, D, F):
+    w = custom(B, L, H, D, F, dtype="f32")
+    inp = make_inputs(w)
+    out, y = run_library(w, inp)
+    out_ref, y_ref = oracle_full(w, inp)
+    check_parity(w, out, y, out_ref, y_ref)
+
+
+@pytest.mark.parametrize("B,L,H,D,F", [(1, 256, 1, 16, 40), (2, 12288, 2, 8, 6145),
+                                       (1, 65536, 2, 8, 8192), (1, 3072, 3, 5, 1)])
+def test_shape_sweep_bf16(B, L, H, D, F):
+    w = custom(B, L, H, D, F, dtype="bf16")
+    inp = make_inputs(w)
+    out, y = run_library(w, inp)
+    out_ref, y_ref = oracle_full(w, inp)
+    check_parity(w, out, y, out_ref, y_ref)
+
+
+def test_zero_gate_gives_layernorm_of_x():
+    w = custom(2, 4096, 4, 16, 2049, dtype="f32")
+    inp = make_inputs(w)
+    inp["G"].zero_()
+    out, y = run_library(w, inp)
+    assert torch.count_nonzero(out) == 0
+    ref = torch.nn.functional.layer_norm(inp["x"].double(), (w.C,), inp["gamma"].double(),
+                                         inp["beta"].double(), eps=float(np.float32(w.eps)))
+    assert float((y.double() - ref).abs().max()) < 1e-5
+
+
+def test_repeat_runs_are_bitwise_identical():
+    w = WORKLOADS["bf16_long"]
+    inp = make_inputs(w)
+    out1, y1 = run_library(w, inp)
+    out2, y2 = run_library(w, inp)
+    assert torch.equal(out1, out2) and torch.equal(y1, y2)
+
+
+def test_host_buffer_entry_point_matches_device_entry_point():
+    from sub_quadratic_attention_b200.binding import SpectreMix
+
+    w = WORKLOADS["fp32_mid"]
+    inp = make_inputs(w)
+    _, y_dev = run_library(w, inp, debug=False)
+    pinned = {k: v.pin_memory() for k, v in inp.items()}
+    y_host = torch.empty_like(pinned["x"]).pin_memory()
+    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps) as mix:
+        for _ in range(2):
+            mix.run_host(pinned["q"], pinned["k"], pinned["v"], pinned["x"], pinned["G"],
+                         pinned["gamma"], pinned["beta"], y_host)
+            torch.cuda.synchronize()
+            assert torch.equal(y_host, y_dev)
+
+
+def test_run_rejects_misaligned_and_null_pointers():
+    from sub_quadratic_attention_b200 import binding as b
+
+    w = WORKLOADS["tiny_fp32"]
+    d = {k: v.cuda() for k, v in make_inputs(w).items()}
+    y = torch.empty_like(d["x"])
+    h = b.spectre_mix_create(w.B, w.L, w.H, w.D, w.F, b.SPECTRE_F32, w.eps)
+    try:
+        args = [d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y]
+        assert b.spectre_mix_run_status(h, *args) == b.SPECTRE_OK
+        bad = list(args)
+        bad[0] = d["q"].data_ptr() + 4
+        assert b.spectre_mix_run_status(h, *bad) == b.SPECTRE_ERR_ALIGN
+        bad = list(args)
+        bad[7] = 0
+        assert b.spectre_mix_run_status(h, *bad) == b.SPECTRE_ERR_ARG
+        torch.cuda.synchronize()
+    finally:
+        b.spectre_mix_destroy(h)
