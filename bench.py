@@ -259,6 +259,10 @@ def native_arm(args, w, rank, world, local_rank):
     sampler.start()
     time.sleep(0.05)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for ev in events:  # torch creates the CUDA event on its first record
+        for e in ev:
+            e.record(stream)
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     t_host0 = time.perf_counter()
