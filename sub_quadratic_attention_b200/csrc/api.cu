@@ -27,8 +27,8 @@ struct spectre_mix_s {
     float2 *A, *P;
     size_t table_bytes, ws_bytes;
     // geometry
-    int CT, TB;          // row pass
     int T2C, ZS;         // inverse row pass
+    int inv_reg;         // register-resident LayerNorm variant
     // staging for spectre_mix_run_host, allocated on first use
     void *stage;
     size_t stage_bytes;
@@ -149,13 +149,19 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     h->R = R; h->M = M; h->NF = NF;
 
     // ---- geometry
-    h->CT = C >= 64 ? 64 : (int)align_up((size_t)C, 2);
-    int tpr = h->CT / 2;
-    int TB = 256 / tpr;
-    while (TB > 1 && (size_t)NF * TB * (h->CT + 4) * sizeof(float2) > 96 * 1024) TB /= 2;
-    h->TB = TB;
-    int T2C = 8;
-    while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
+    // inverse row pass: register-resident LayerNorm when a block of
+    // T2C x ceil(C/2) <= 1024 threads covers the channels; else the
+    // shared-memory variant (R rows x T2C x padded C floats per block)
+    const int CP = (C + 1) / 2;
+    h->inv_reg = (R <= 16 && CP <= 1024) ? 1 : 0;
+    int T2C;
+    if (h->inv_reg) {
+        T2C = 1;
+        while (T2C < 8 && T2C * 2 * CP <= (CP > 512 ? 1024 : 512) && T2C * 2 <= M) T2C *= 2;
+    } else {
+        T2C = 8;
+        while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
+    }
     h->T2C = T2C;
     h->ZS = ZS;
 
@@ -177,8 +183,8 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
                 size_t base = align_up(host.size(), 2);
                 host.resize(base);
                 offs[d][p] = base;
-                for (int kk = 0; kk < ns; kk++)
-                    for (int rr = 0; rr < r; rr++) {
+                for (int rr = 0; rr < r; rr++)
+                    for (int kk = 0; kk < ns; kk++) {
                         long long e = (long long)kk * rr;
                         double ang = -2.0 * M_PI * (double)e / (double)(ns * r);
                         host.push_back(make_float2((float)std::cos(ang), (float)std::sin(ang)));
@@ -246,7 +252,6 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
     fa.A = h->A;
     fa.twL = h->twL;
     fa.B = h->B; fa.L = h->L; fa.M = h->M; fa.C = h->C;
-    fa.CT = h->CT; fa.TB = h->TB;
     fa.vec2 = (h->C % 2 == 0) ? 1 : 0;
     cudaError_t e = mark(0);
     if (e == cudaSuccess) e = launch_rows_fwd(h->R, h->dtype, fa, s);
@@ -266,6 +271,8 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
     ia.P = h->P; ia.x = x; ia.gamma = gamma; ia.beta = beta; ia.y = y; ia.out_f32 = out_f32;
     ia.B = h->B; ia.L = h->L; ia.M = h->M; ia.C = h->C;
     ia.T2C = h->T2C; ia.ZS = h->ZS; ia.eps = h->eps;
+    ia.reg_variant = h->inv_reg;
+    ia.vec2 = (h->C % 2 == 0) ? 1 : 0;
     e = mark(2);
     if (e == cudaSuccess) e = launch_rows_inv_ln(h->R, h->dtype, ia, s);
     if (e == cudaSuccess) e = mark(3);

@@ -26,6 +26,9 @@ template <> struct Elem<float> {
         return __ldg(reinterpret_cast<const float2 *>(p));
     }
     __device__ __forceinline__ static void store(float *p, float v) { *p = v; }
+    __device__ __forceinline__ static void store2(float *p, float v0, float v1) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v0, v1);
+    }
 };
 template <> struct Elem<__nv_bfloat16> {
     __device__ __forceinline__ static float load(const __nv_bfloat16 *p) {
@@ -35,6 +38,9 @@ template <> struct Elem<__nv_bfloat16> {
         return __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p)));
     }
     __device__ __forceinline__ static void store(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+    __device__ __forceinline__ static void store2(__nv_bfloat16 *p, float v0, float v1) {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v0, v1);
+    }
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -45,24 +51,27 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------------------
 // row pass: A[sig][b][c][f1][t2] = w_L^{f1 t2} sum_{t1} w_R^{f1 t1} sig[b][t1 M + t2][c]
-// Block: (CT/2) x TB threads; thread (tx, ty) owns channels 2tx, 2tx+1 of the
-// tile at t2 = tile*TB + ty, packed as one complex signal (c0 + i c1).
+// Block: 256 threads = 8 warps over 8 t2 values x 32 channel pairs; a warp
+// covers 4 consecutive t2 x 8 consecutive channel pairs, lane = tl + 4 cpl.
+// Each thread owns channels c0 = 2 cp, c0 + 1 at one t2, packed as one complex
+// signal c0 + i c1.  Its 16-row loads are 32-byte segments per warp-row
+// (8 channel pairs) and its stores are 32-byte segments (4 consecutive t2) of
+// A, straight from registers.
 // ---------------------------------------------------------------------------
 template <int R, typename T>
-__global__ void __launch_bounds__(256) spectre_rows_fwd(RowsFwdArgs a) {
+__global__ void __launch_bounds__(256, R <= 16 ? 3 : 1) spectre_rows_fwd(RowsFwdArgs a) {
     constexpr int NF = R / 2 + 1;
-    extern __shared__ float4 smem_f4[];
-    float2 *stage = reinterpret_cast<float2 *>(smem_f4);  // [NF][TB][CT + 4]
-    const int CT = a.CT, TB = a.TB, CTP = a.CT + 4;
-    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t2 = blockIdx.x * 8 + (warp & 1) * 4 + (lane & 3);
+    const int cp = blockIdx.y * 32 + (warp >> 1) * 8 + (lane >> 2);
     const int b = blockIdx.z;
-    const int t2 = blockIdx.x * TB + ty;
-    const int c0 = blockIdx.y * CT + 2 * tx;
+    const int c0 = 2 * cp;
     const bool live = (t2 < a.M) && (c0 < a.C);
-    const bool has1 = (c0 + 1 < a.C);
+    const bool has1 = live && (c0 + 1 < a.C);
     const size_t rowstride = (size_t)a.M * a.C;
-    const int nthr = blockDim.x * blockDim.y;
-    const int tid = ty * blockDim.x + tx;
+    const size_t plane = (size_t)a.B * a.C * NF * a.M;
+    float2 *dst0 = a.A + ((size_t)b * a.C + c0) * NF * a.M + t2;
+    float2 *dst1 = dst0 + (size_t)NF * a.M;
 
 #pragma unroll 1
     for (int sig = 0; sig < 3; sig++) {
@@ -85,33 +94,23 @@ __global__ void __launch_bounds__(256) spectre_rows_fwd(RowsFwdArgs a) {
             for (int t1 = 0; t1 < R; t1++) z[t1] = make_float2(0.f, 0.f);
         }
         Dft<R>::run(z);
-        // separate the two real channels, twiddle by w_L^{f1 t2}, stage
+        // separate the two real channels, twiddle by w_L^{f1 t2}, store
+        if (live) {
 #pragma unroll
-        for (int f1 = 0; f1 < NF; f1++) {
-            float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
-            float2 xa = cscale(cadd(zf, zc), 0.5f);
-            float2 d = csub(zf, zc);
-            float2 xb = make_float2(0.5f * d.y, -0.5f * d.x);
-            if (f1 > 0 && live) {
-                float2 w = __ldg(a.twL + f1 * t2);
-                xa = cmul(xa, w);
-                xb = cmul(xb, w);
+            for (int f1 = 0; f1 < NF; f1++) {
+                float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
+                float2 xa = cscale(cadd(zf, zc), 0.5f);
+                float2 d = csub(zf, zc);
+                float2 xb = make_float2(0.5f * d.y, -0.5f * d.x);
+                if (f1 > 0) {
+                    float2 w = __ldg(a.twL + f1 * t2);
+                    xa = cmul(xa, w);
+                    xb = cmul(xb, w);
+                }
+                dst0[sig * plane + (size_t)f1 * a.M] = xa;
+                if (has1) dst1[sig * plane + (size_t)f1 * a.M] = xb;
             }
-            *reinterpret_cast<float4 *>(stage + (f1 * TB + ty) * CTP + 2 * tx) =
-                make_float4(xa.x, xa.y, xb.x, xb.y);
         }
-        __syncthreads();
-        // store segments of TB consecutive t2 per (c, f1)
-        const int total = CT * NF * TB;
-        float2 *dst = a.A + (size_t)(sig * a.B + b) * a.C * NF * a.M;
-        for (int i = tid; i < total; i += nthr) {
-            int tl = i % TB, rest = i / TB;
-            int cl = rest % CT, f1 = rest / CT;
-            int c = blockIdx.y * CT + cl, tt = blockIdx.x * TB + tl;
-            if (c < a.C && tt < a.M)
-                dst[((size_t)c * NF + f1) * a.M + tt] = stage[(f1 * TB + tl) * CTP + cl];
-        }
-        __syncthreads();
     }
 }
 
@@ -121,7 +120,8 @@ __global__ void __launch_bounds__(256) spectre_rows_fwd(RowsFwdArgs a) {
 __device__ __forceinline__ int spad(int i) { return i + (i >> 4); }
 
 // One in-place Stockham pass over shared memory:
-//   butterfly bf < M/R reads buf[bf + r M/R], twiddles by w_{Ns R}^{(bf mod Ns) r},
+//   butterfly bf < M/R reads buf[bf + r M/R], twiddles by w_{Ns R}^{(bf mod Ns) r}
+//   (table entry tw[r Ns + bf mod Ns], so a warp's loads are contiguous),
 //   and writes buf[(bf / Ns) Ns R + (bf mod Ns) + r Ns].
 template <int R, int M, int NT, int NS>
 __device__ __forceinline__ void smem_pass(float2 *buf, const float2 *__restrict__ tw, int j) {
@@ -143,9 +143,9 @@ __device__ __forceinline__ void smem_pass(float2 *buf, const float2 *__restrict_
         if (NBF % NT == 0 || bf < NBF) {
             int kk = bf % NS;
             if (NS > 1) {
-                const float2 *t = tw + kk * R;
+                const float2 *t = tw + kk;
 #pragma unroll
-                for (int r = 1; r < R; r++) v[i][r] = cmul(v[i][r], __ldg(t + r));
+                for (int r = 1; r < R; r++) v[i][r] = cmul(v[i][r], __ldg(t + r * NS));
             }
             Dft<R>::run(v[i]);
             int idxD = (bf / NS) * NS * R + kk;
@@ -167,6 +167,10 @@ template <int M, int NT, int D, int P, int PEND> struct MidPasses {
     }
 };
 
+// Where the running product S = Q conj(K) G' / L lives between the three
+// forward transforms of a slice.
+enum SliceProduct { kProdSmem = 0, kProdRegs = 1, kProdGlobal = 2 };
+
 template <int M> struct SliceCfg {
     static constexpr RadList S = make_schedule(M);
     static constexpr int NP = S.n;
@@ -175,8 +179,14 @@ template <int M> struct SliceCfg {
     static constexpr int NT = M / RL;                      // threads per slice
     static constexpr int SPB = NT >= 256 ? 1 : 256 / NT;   // slices per block
     static constexpr int THREADS = NT * SPB;
-    static constexpr int BUF = NP >= 2 ? (M + M / 16) : 0; // float2 per slice
-    static constexpr bool S_IN_REGS = NT <= 512;
+    static constexpr int BUF = NP >= 2 ? (M + M / 16) : 0; // float2 per slice (padded)
+    static constexpr int PROD = (BUF + M) * SPB * 8 <= 72 * 1024 ? kProdSmem
+                              : (NT <= 512 ? kProdRegs : kProdGlobal);
+    static constexpr int SMEM = (BUF + (PROD == kProdSmem ? M : 0)) * SPB * 8;
+    // blocks per SM the register budget must allow
+    static constexpr int MINB0 = PROD == kProdSmem ? (SMEM > 0 ? (200 * 1024) / SMEM : 4) : 1;
+    static constexpr int MINB = MINB0 > 4 ? 4 : MINB0;
+    static constexpr int MINB_C = MINB < 1 ? 1 : (MINB * THREADS > 2048 ? 2048 / THREADS : MINB);
 };
 
 // Forward M-point transform of one slice of A.  On return thread j holds
@@ -217,9 +227,9 @@ __device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bo
         constexpr int RL = Cfg::RL;
 #pragma unroll
         for (int r = 0; r < RL; r++) x[r] = buf[spad(j + r * NT)];
-        const float2 *t = tb.tw[0][NP - 1] + j * RL;
+        const float2 *t = tb.tw[0][NP - 1] + j;
 #pragma unroll
-        for (int r = 1; r < RL; r++) x[r] = cmul(x[r], __ldg(t + r));
+        for (int r = 1; r < RL; r++) x[r] = cmul(x[r], __ldg(t + r * NT));
         Dft<RL>::run(x);
     }
 }
@@ -269,7 +279,7 @@ __device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL]
 #pragma unroll
                 for (int r = 0; r < R; r++) v[r] = buf[spad(bf + r * NBF)];
 #pragma unroll
-                for (int r = 1; r < R; r++) v[r] = cmul(v[r], __ldg(tw + bf * R + r));
+                for (int r = 1; r < R; r++) v[r] = cmul(v[r], __ldg(tw + bf + r * NBF));
                 Dft<R>::run(v);
                 if (live) {
 #pragma unroll
@@ -285,13 +295,14 @@ __device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL]
 }
 
 template <int M>
-__global__ void __launch_bounds__(SliceCfg<M>::THREADS) spectre_slices(SliceArgs a) {
+__global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spectre_slices(SliceArgs a) {
     using Cfg = SliceCfg<M>;
-    constexpr int NT = Cfg::NT, RL = Cfg::RL;
+    constexpr int NT = Cfg::NT, RL = Cfg::RL, PROD = Cfg::PROD;
     extern __shared__ float4 smem_f4[];
     const int sl = threadIdx.x / NT;
     const int j = threadIdx.x % NT;
     float2 *buf = reinterpret_cast<float2 *>(smem_f4) + sl * Cfg::BUF;
+    float2 *sbuf = reinterpret_cast<float2 *>(smem_f4) + Cfg::SPB * Cfg::BUF + sl * M;
     const long long sid = (long long)blockIdx.x * Cfg::SPB + sl;
     const bool live = sid < a.nslices;
     const int NF = a.R / 2 + 1;
@@ -307,46 +318,38 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS) spectre_slices(SliceArgs
 
     float2 x[RL];
     float2 s[RL];
-    // q: S = Q * G' / L on this thread's bins f = f1 + R (j + r NT)
+    // each thread owns bins f = f1 + R (j + r NT), r < RL, of the product;
+    // with kProdGlobal the slice's P row holds S until it is overwritten
+    auto put = [&](int r, float2 v) {
+        if constexpr (PROD == kProdSmem) sbuf[j + r * NT] = v;
+        else if constexpr (PROD == kProdRegs) s[r] = v;
+        else { if (live) dstP[j + r * NT] = v; }
+    };
+    auto get = [&](int r) -> float2 {
+        if constexpr (PROD == kProdSmem) return sbuf[j + r * NT];
+        else if constexpr (PROD == kProdRegs) return s[r];
+        else return live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
+    };
+
+    // q: S = Q * G' / L
     slice_forward<M>(srcA, live, buf, a.tabs, j, x);
 #pragma unroll
     for (int r = 0; r < RL; r++) {
         int f = f1 + a.R * (j + r * NT);
         int ff = min(f, a.L - f);
         float g = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
-        s[r] = cscale(x[r], g);
-    }
-    if constexpr (!Cfg::S_IN_REGS) {
-        // park S in this slice's P row (rewritten at the end)
-        if (live) {
-#pragma unroll
-            for (int r = 0; r < RL; r++) dstP[j + r * NT] = s[r];
-        }
+        put(r, cscale(x[r], g));
     }
     if constexpr (Cfg::NP >= 2) __syncthreads();
     // k: S *= conj(K)
     slice_forward<M>(srcA + sig_stride, live, buf, a.tabs, j, x);
-    if constexpr (!Cfg::S_IN_REGS) {
 #pragma unroll
-        for (int r = 0; r < RL; r++) s[r] = live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int r = 0; r < RL; r++) s[r] = cmulc(s[r], x[r]);
-    if constexpr (!Cfg::S_IN_REGS) {
-        if (live) {
-#pragma unroll
-            for (int r = 0; r < RL; r++) dstP[j + r * NT] = s[r];
-        }
-    }
+    for (int r = 0; r < RL; r++) put(r, cmulc(get(r), x[r]));
     if constexpr (Cfg::NP >= 2) __syncthreads();
     // v: O = S * V
     slice_forward<M>(srcA + 2 * sig_stride, live, buf, a.tabs, j, x);
-    if constexpr (!Cfg::S_IN_REGS) {
 #pragma unroll
-        for (int r = 0; r < RL; r++) s[r] = live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int r = 0; r < RL; r++) x[r] = cmul(s[r], x[r]);
+    for (int r = 0; r < RL; r++) x[r] = cmul(get(r), x[r]);
     slice_inverse_store<M>(x, buf, a.tabs, j, live, dstP, a.twL, f1);
 }
 
@@ -435,23 +438,137 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// inverse row pass + residual + LayerNorm, register-resident variant.
+// Block: T2C x CP threads (CP = ceil(C/2) channel pairs, T2C t2 values,
+// thread = tl + T2C * cp).  Each thread inverts its channel pair's R-point
+// spectrum at one t2 and keeps the R x 2 values of z = out + x in registers;
+// the LayerNorm statistics of the R * T2C token rows are reduced with warp
+// shuffles and one shared-memory stage, in two passes (mean, then the mean
+// of squared deviations), in a fixed order.
+// ---------------------------------------------------------------------------
+template <int R, typename T, bool DEBUG_OUT>
+__global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
+    constexpr int NF = R / 2 + 1;
+    extern __shared__ float4 smem_f4[];
+    float *part = reinterpret_cast<float *>(smem_f4);   // [nwarps][T2C][R], then stat[2][T2C][R]
+    const int T2C = a.T2C;
+    const int nthr = blockDim.x;
+    const int nwarps = nthr >> 5;
+    float *stat = part + nwarps * T2C * R;               // [T2C][R]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tl = tid & (T2C - 1), cp = tid / T2C;
+    const int b = blockIdx.y;
+    const int t2 = blockIdx.x * T2C + tl;
+    const int c0 = 2 * cp;
+    const bool live = (t2 < a.M) && (c0 < a.C);
+    const bool has1 = live && (c0 + 1 < a.C);
+    float z0[R], z1[R];
+    {
+        float2 Z[R];
+        const float2 *pa = a.P + ((size_t)b * a.C + c0) * NF * a.M + t2;
+        const float2 *pb = pa + (size_t)NF * a.M;
+        const float2 zero = make_float2(0.f, 0.f);
+        float2 a0 = live ? __ldg(pa) : zero, aN = live ? __ldg(pa + (size_t)(R / 2) * a.M) : zero;
+        float2 b0 = has1 ? __ldg(pb) : zero, bN = has1 ? __ldg(pb + (size_t)(R / 2) * a.M) : zero;
+        Z[0] = make_float2(a0.x, -b0.x);
+        Z[R / 2] = make_float2(aN.x, -bN.x);
+#pragma unroll
+        for (int f1 = 1; f1 < R / 2; f1++) {
+            float2 pv = live ? __ldg(pa + (size_t)f1 * a.M) : zero;
+            float2 qv = has1 ? __ldg(pb + (size_t)f1 * a.M) : zero;
+            Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
+            Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
+        }
+        Dft<R>::run(Z);
+#pragma unroll
+        for (int t1 = 0; t1 < R; t1++) {
+            z0[t1] = Z[t1].x;
+            z1[t1] = -Z[t1].y;
+        }
+    }
+    const T *x = static_cast<const T *>(a.x);
+    const size_t tok0 = (size_t)b * a.L + t2;
+    const size_t rowstep = (size_t)a.M * a.C;
+    const T *xp = x + tok0 * a.C + c0;
+    float s[R];
+#pragma unroll
+    for (int t1 = 0; t1 < R; t1++) {
+        if (DEBUG_OUT && live) {
+            float *op = a.out_f32 + tok0 * a.C + c0 + t1 * rowstep;
+            if (has1 && a.vec2)
+                *reinterpret_cast<float2 *>(op) = make_float2(z0[t1], z1[t1]);
+            else {
+                op[0] = z0[t1];
+                if (has1) op[1] = z1[t1];
+            }
+        }
+        if (has1 && a.vec2) {
+            float2 xv = Elem<T>::load2(xp + t1 * rowstep);
+            z0[t1] += xv.x;
+            z1[t1] += xv.y;
+        } else {
+            z0[t1] = live ? z0[t1] + Elem<T>::load(xp + t1 * rowstep) : 0.f;
+            z1[t1] = has1 ? z1[t1] + Elem<T>::load(xp + t1 * rowstep + 1) : 0.f;
+        }
+        s[t1] = z0[t1] + z1[t1];
+    }
+    const float invC = 1.0f / (float)a.C;
+    // two reductions over the channels of each row: sum(z), then sum((z - mean)^2);
+    // stat[0][.] holds the means, stat[1][.] the variances
+#pragma unroll 1
+    for (int pass = 0; pass < 2; pass++) {
+        if (pass == 1) {
+#pragma unroll
+            for (int t1 = 0; t1 < R; t1++) {
+                const float mu = stat[tl * R + t1];
+                float d0 = z0[t1] - mu, d1 = z1[t1] - mu;
+                s[t1] = live ? fmaf(d0, d0, has1 ? d1 * d1 : 0.f) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int t1 = 0; t1 < R; t1++)
+            for (int o = T2C; o < 32; o <<= 1) s[t1] += __shfl_xor_sync(0xffffffffu, s[t1], o);
+        if (lane < T2C) {
+#pragma unroll
+            for (int t1 = 0; t1 < R; t1++) part[(warp * T2C + tl) * R + t1] = s[t1];
+        }
+        __syncthreads();
+        for (int i = tid; i < T2C * R; i += nthr) {
+            float acc = 0.f;
+            for (int w = 0; w < nwarps; w++) acc += part[w * T2C * R + i];
+            stat[pass * T2C * R + i] = acc * invC;
+        }
+        __syncthreads();
+    }
+    T *y = static_cast<T *>(a.y);
+    T *yp = y + tok0 * a.C + c0;
+    const float g0 = live ? __ldg(a.gamma + c0) : 0.f, be0 = live ? __ldg(a.beta + c0) : 0.f;
+    const float g1 = has1 ? __ldg(a.gamma + c0 + 1) : 0.f, be1 = has1 ? __ldg(a.beta + c0 + 1) : 0.f;
+#pragma unroll
+    for (int t1 = 0; t1 < R; t1++) {
+        const float mu = stat[tl * R + t1];
+        const float rstd = rsqrtf(stat[T2C * R + tl * R + t1] + a.eps);
+        const float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
+        const float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
+        if (has1 && a.vec2) {
+            Elem<T>::store2(yp + t1 * rowstep, y0, y1);
+        } else if (live) {
+            Elem<T>::store(yp + t1 * rowstep, y0);
+            if (has1) Elem<T>::store(yp + t1 * rowstep + 1, y1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
 template <int R>
 static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a, cudaStream_t s) {
-    constexpr int NF = R / 2 + 1;
-    dim3 block(a.CT / 2, a.TB);
-    dim3 grid((a.M + a.TB - 1) / a.TB, (a.C + a.CT - 1) / a.CT, a.B);
-    size_t smem = (size_t)NF * a.TB * (a.CT + 4) * sizeof(float2);
-    if (dtype == 0) {
-        auto k = spectre_rows_fwd<R, float>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, block, smem, s>>>(a);
-    } else {
-        auto k = spectre_rows_fwd<R, __nv_bfloat16>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, block, smem, s>>>(a);
-    }
+    dim3 grid((a.M + 7) / 8, (a.C + 63) / 64, a.B);
+    if (dtype == 0)
+        spectre_rows_fwd<R, float><<<grid, 256, 0, s>>>(a);
+    else
+        spectre_rows_fwd<R, __nv_bfloat16><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -468,7 +585,7 @@ cudaError_t launch_rows_fwd(int R, int dtype, const RowsFwdArgs &a, cudaStream_t
 template <int M>
 static cudaError_t slices_M(const SliceArgs &a, cudaStream_t s) {
     using Cfg = SliceCfg<M>;
-    size_t smem = (size_t)Cfg::BUF * Cfg::SPB * sizeof(float2);
+    size_t smem = (size_t)Cfg::SMEM;
     long long nblk = (a.nslices + Cfg::SPB - 1) / Cfg::SPB;
     auto k = spectre_slices<M>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -480,7 +597,7 @@ template <int M> static void slice_geom_M(int *nt, int *spb, size_t *smem) {
     using Cfg = SliceCfg<M>;
     *nt = Cfg::NT;
     *spb = Cfg::SPB;
-    *smem = (size_t)Cfg::BUF * Cfg::SPB * sizeof(float2);
+    *smem = (size_t)Cfg::SMEM;
 }
 
 #define SPECTRE_SLICE_LENGTHS(X)                                                              \
@@ -520,6 +637,17 @@ void slice_geometry(int M, int *nt, int *spb, size_t *smem) {
 
 template <int R, typename T>
 static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
+    if constexpr (R <= 16) if (a.reg_variant) {
+        dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
+        const int CP = (a.C + 1) / 2;
+        const int threads = ((a.T2C * CP + 31) / 32) * 32;
+        size_t smem = (size_t)((threads / 32) * a.T2C * R + 2 * a.T2C * R) * sizeof(float);
+        if (a.out_f32)
+            spectre_rows_inv_ln_reg<R, T, true><<<grid, threads, smem, s>>>(a);
+        else
+            spectre_rows_inv_ln_reg<R, T, false><<<grid, threads, smem, s>>>(a);
+        return cudaGetLastError();
+    }
     dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
     size_t smem = (size_t)R * a.T2C * a.ZS * sizeof(float);
     if (a.out_f32) {

@@ -26,7 +26,7 @@ constexpr int kMaxPasses = 6;
 // Per-pass twiddle tables of the M-point slice transforms.  Pass p of
 // direction d (0 = forward radix order, 1 = reversed) with radix R_p and
 // stride Ns_p (product of the earlier radices) uses
-//   tw[d][p][k * R_p + r] = exp(-2 pi i k r / (Ns_p R_p)),  k < Ns_p, r < R_p.
+//   tw[d][p][r * Ns_p + k] = exp(-2 pi i k r / (Ns_p R_p)),  k < Ns_p, r < R_p.
 struct SliceTables {
     const float2 *tw[2][kMaxPasses];
 };
@@ -36,7 +36,6 @@ struct RowsFwdArgs {
     float2 *A;            // [3][B][C][R/2+1][M]
     const float2 *twL;    // exp(-2 pi i e / L), e in [0, L/2]
     int B, L, M, C;
-    int CT, TB;           // channel tile, t2 tile
     int vec2;             // C even: load channel pairs as one vector
 };
 
@@ -59,6 +58,8 @@ struct RowsInvArgs {
     float *out_f32;       // nullable
     int B, L, M, C;
     int T2C, ZS;          // t2 values per block, padded row stride of the z buffer
+    int reg_variant;      // 1: register-resident LayerNorm (R <= 16, C <= 2048)
+    int vec2;             // C even: channel pairs as one vector
     float eps;
 };
 
