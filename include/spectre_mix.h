@@ -57,8 +57,12 @@ enum spectre_status {
     SPECTRE_ERR_ALIGN = -3,         /* a tensor pointer is not 16-byte aligned */
     SPECTRE_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
     SPECTRE_ERR_NOMEM = -5,         /* device or host allocation failed */
-    SPECTRE_ERR_DEVICE = -6         /* no usable sm_100 device, or wrong current device */
+    SPECTRE_ERR_DEVICE = -6,        /* no usable sm_100 device, or wrong current device */
+    SPECTRE_ERR_SCRATCH = -7        /* problem too large for the no-allocation scratch */
 };
+
+/* Size of the fixed device scratch behind spectre_mix_run_noalloc. */
+#define SPECTRE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
 /*
  * Create a plan for one problem shape.  Validates the shape, picks the
@@ -124,6 +128,39 @@ int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k,
                              const void *v, const void *x, const float *G,
                              const float *gamma, const float *beta, void *y,
                              void *const *events, void *stream);
+
+/*
+ * One mix that allocates nothing.  The pages have no counterpart: this entry
+ * point exists for callers that may not call cudaMalloc -- for instance code
+ * running inside a framework whose caching allocator owns the device memory
+ * and forbids side allocations, or a latency-critical loop that cannot accept
+ * the device-wide synchronisation cudaMalloc and cudaFree can imply.
+ *
+ * Same operation, shapes, types and pointer rules as spectre_mix_run, with the
+ * plan arguments of spectre_mix_create passed on every call (no handle).  The
+ * caller still provides every input and output.  Instead of a workspace
+ * allocated per plan, the call uses one fixed device array of
+ * SPECTRE_NOALLOC_SCRATCH_BYTES (64 MiB) built into the library; every GPU
+ * that loads the library holds that array until the process exits.  Twiddle
+ * tables are rebuilt in the scratch by a small kernel on each call; the rest
+ * of the scratch is fully overwritten before it is read, so nothing carries
+ * over from the previous call.
+ *
+ *   Returns SPECTRE_ERR_SCRATCH when the tables plus the workspace of this
+ *   shape (4 * B * C * (R/2+1) * M * 8 bytes, see spectre_mix_plan_info)
+ *   exceed the scratch; other errors as spectre_mix_create/spectre_mix_run.
+ *
+ * The first call on a device looks up the scratch's device address and loads
+ * constant twiddles (synchronous); make that first call before any stream
+ * capture.  All calls on a device share the one scratch array, so calls that
+ * overlap on the GPU (other streams, other host threads) race: serialise them.
+ * Asynchronous otherwise: returns after the launches are queued on `stream`.
+ */
+int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype,
+                            float eps, const void *q, const void *k,
+                            const void *v, const void *x, const float *G,
+                            const float *gamma, const float *beta, void *y,
+                            void *stream);
 
 /* Free the handle, its tables, workspace and staging buffers.  NULL-safe.
  * Synchronises the device the handle lives on before freeing. */

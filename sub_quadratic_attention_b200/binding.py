@@ -23,6 +23,10 @@ SPECTRE_ERR_ALIGN = -3
 SPECTRE_ERR_CUDA = -4
 SPECTRE_ERR_NOMEM = -5
 SPECTRE_ERR_DEVICE = -6
+SPECTRE_ERR_SCRATCH = -7
+
+# fixed device scratch behind spectre_mix_run_noalloc (SPECTRE_NOALLOC_SCRATCH_BYTES)
+SPECTRE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 # every entry point the header declares, with its ctypes signature
 _vp = ctypes.c_void_p
@@ -33,6 +37,7 @@ SIGNATURES = {
     "spectre_mix_run_debug": (_i, [_vp] * 11),
     "spectre_mix_run_host": (_i, [_vp] * 10),
     "spectre_mix_run_profiled": (_i, [_vp] * 11),
+    "spectre_mix_run_noalloc": (_i, [_i] * 6 + [ctypes.c_float] + [_vp] * 9),
     "spectre_mix_destroy": (_i, [_vp]),
     "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
     "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
@@ -135,6 +140,21 @@ def spectre_mix_run_profiled(h: int, q, k, v, x, G, gamma, beta, y, events, stre
                                          _ptr(gamma), _ptr(beta), _ptr(y),
                                          ctypes.cast(arr, _vp), _stream(stream)),
            "spectre_mix_run_profiled")
+
+
+def spectre_mix_run_noalloc_status(B: int, L: int, H: int, D: int, F: int, dtype: int, eps: float,
+                                   q, k, v, x, G, gamma, beta, y, stream=None) -> int:
+    """One mix with no device allocation (the library's fixed 64 MiB scratch);
+    for callers that may not call cudaMalloc.  Returns the raw status."""
+    return _lib.spectre_mix_run_noalloc(B, L, H, D, F, dtype, eps, _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(x), _ptr(G), _ptr(gamma), _ptr(beta), _ptr(y),
+                                        _stream(stream))
+
+
+def spectre_mix_run_noalloc(B: int, L: int, H: int, D: int, F: int, dtype: int, eps: float,
+                            q, k, v, x, G, gamma, beta, y, stream=None) -> None:
+    _check(spectre_mix_run_noalloc_status(B, L, H, D, F, dtype, eps, q, k, v, x, G, gamma, beta,
+                                          y, stream), "spectre_mix_run_noalloc")
 
 
 def spectre_mix_destroy(h: Optional[int]) -> None:

@@ -116,6 +116,7 @@ const char *spectre_mix_error_string(int code) {
     case SPECTRE_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
     case SPECTRE_ERR_NOMEM: return "out of memory";
     case SPECTRE_ERR_DEVICE: return "no usable sm_100 device, or the handle's device is not current";
+    case SPECTRE_ERR_SCRATCH: return "problem needs more than the 64 MiB no-allocation scratch holds";
     default: return "unknown status";
     }
 }
@@ -346,6 +347,113 @@ int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k, const vo
         cudaGetLastError();
         return cuda_status(e);
     }
+    return SPECTRE_OK;
+}
+
+int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float eps, const void *q,
+                            const void *k, const void *v, const void *x, const float *G,
+                            const float *gamma, const float *beta, void *y, void *stream) {
+    // the same validation as spectre_mix_create and spectre_mix_run
+    if (B < 1 || B > 65535 || H < 1 || D < 1 || L < 1) return SPECTRE_ERR_ARG;
+    if (dtype != SPECTRE_F32 && dtype != SPECTRE_BF16) return SPECTRE_ERR_ARG;
+    if (!(eps > 0.0f) || !std::isfinite(eps)) return SPECTRE_ERR_ARG;
+    if ((long long)H * D > (1 << 20)) return SPECTRE_ERR_ARG;
+    int R = 0, M = 0;
+    if (!choose_split(L, &R, &M)) return SPECTRE_ERR_UNSUPPORTED_L;
+    if (F < 1 || F > L / 2 + 1) return SPECTRE_ERR_ARG;
+    const int C = H * D;
+    const int NF = R / 2 + 1;
+    const int ZS = (int)align_up((size_t)C, 32) + 16;
+    if ((size_t)R * ZS * sizeof(float) > 227 * 1024) return SPECTRE_ERR_ARG;
+    if (!q || !k || !v || !x || !G || !gamma || !beta || !y) return SPECTRE_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(x) || !aligned16(G) ||
+        !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
+        return SPECTRE_ERR_ALIGN;
+
+    // scratch layout: twiddle tables (as spectre_mix_create lays them out),
+    // then A [3][B][C][NF][M] and P [B][C][NF][M], all fp32 complex
+    const RadList sch = make_schedule(M);
+    TableSegs segs;
+    segs.n = 0;
+    size_t n_tab = (size_t)L / 2 + 1;
+    segs.seg[segs.n++] = TableSeg{0, (long long)n_tab, 0, (long long)L};
+    for (int d = 0; d < 2; d++) {
+        int ns = 1;
+        for (int p = 0; p < sch.n; p++) {
+            int r = d == 0 ? sch.r[p] : sch.r[sch.n - 1 - p];
+            if (p > 0) {
+                size_t base = align_up(n_tab, 2);
+                segs.seg[segs.n++] = TableSeg{(long long)base, (long long)ns * r, (long long)ns,
+                                              (long long)ns * r};
+                n_tab = base + (size_t)ns * r;
+            }
+            ns *= r;
+        }
+    }
+    const size_t tab_bytes = align_up(n_tab * sizeof(float2), 256);
+    const size_t slice_elems = (size_t)B * C * NF * M;
+    const size_t need = tab_bytes + 4 * slice_elems * sizeof(float2);
+    if (need > kNoAllocScratchBytes) return SPECTRE_ERR_SCRATCH;
+
+    int dev = -1;
+    int st = check_device(&dev);
+    if (st != SPECTRE_OK) return st;
+    if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
+    void *scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_status(e);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float2 *tw = static_cast<float2 *>(scratch);
+    float2 *A = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + tab_bytes);
+    float2 *P = A + 3 * slice_elems;
+    e = launch_make_tables(tw, segs, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    SliceTables tabs;
+    {
+        int si = 1;
+        for (int d = 0; d < 2; d++)
+            for (int p = 0; p < kMaxPasses; p++)
+                tabs.tw[d][p] = (p > 0 && p < sch.n) ? tw + segs.seg[si++].offset : nullptr;
+    }
+    const int CP = (C + 1) / 2;
+    const int inv_reg = (R <= 16 && CP <= 1024) ? 1 : 0;
+    int T2C;
+    if (inv_reg) {
+        T2C = 1;
+        while (T2C < 8 && T2C * 2 * CP <= (CP > 512 ? 1024 : 512) && T2C * 2 <= M) T2C *= 2;
+    } else {
+        T2C = 8;
+        while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
+    }
+
+    RowsFwdArgs fa;
+    fa.q = q; fa.k = k; fa.v = v; fa.A = A; fa.twL = tw;
+    fa.B = B; fa.L = L; fa.M = M; fa.C = C;
+    fa.vec2 = (C % 2 == 0) ? 1 : 0;
+    e = launch_rows_fwd(R, dtype, fa, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    SliceArgs sa;
+    sa.A = A; sa.P = P; sa.twL = tw; sa.G = G; sa.tabs = tabs;
+    sa.B = B; sa.L = L; sa.R = R; sa.M = M; sa.C = C; sa.D = D; sa.F = F;
+    sa.nbins = L / 2 + 1;
+    sa.nslices = (long long)B * C * NF;
+    sa.invL = 1.0f / (float)L;
+    e = launch_slices(sa, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    RowsInvArgs ia;
+    ia.P = P; ia.x = x; ia.gamma = gamma; ia.beta = beta; ia.y = y; ia.out_f32 = nullptr;
+    ia.B = B; ia.L = L; ia.M = M; ia.C = C;
+    ia.T2C = T2C; ia.ZS = ZS; ia.eps = eps;
+    ia.reg_variant = inv_reg;
+    ia.vec2 = (C % 2 == 0) ? 1 : 0;
+    e = launch_rows_inv_ln(R, dtype, ia, s);
+    if (e != cudaSuccess) return cuda_status(e);
     return SPECTRE_OK;
 }
 

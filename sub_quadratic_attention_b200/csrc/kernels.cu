@@ -11,6 +11,8 @@
 // The index algebra is in kernels.cuh.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "fft_regs.cuh"
 #include "kernels.cuh"
 
@@ -675,6 +677,78 @@ cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStrea
     case 64: return rows_inv_R<64>(dtype, a, s);
     default: return cudaErrorInvalidValue;
     }
+}
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for the entry point that allocates nothing.  The array lives
+// in this module's global memory on every device that loads the library, from
+// module load until process exit.  Host code reaches it only through the
+// address cudaGetSymbolAddress returns for the current device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices];
+}  // namespace
+
+cudaError_t noalloc_scratch(void **ptr) {
+    *ptr = nullptr;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        // once per device, with that device current: the scratch's device
+        // address and the 64-point constant twiddles the R = 64 kernels use
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        float2 w64[64];
+        for (int i = 0; i < 64; i++) {
+            double ang = -2.0 * 3.14159265358979323846 * i / 64.0;
+            w64[i] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+        e = upload_w64(w64);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = addr;
+    }
+    *ptr = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+// Twiddle tables computed on the device (fp64 sincospi, stored fp32), in the
+// layout spectre_mix_create builds on the host.
+__global__ void spectre_make_tables(float2 *base, TableSegs segs) {
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int sgi = 0; sgi < segs.n; sgi++) {
+        const TableSeg &g = segs.seg[sgi];
+        if (i < g.count) {
+            long long e;
+            if (g.ns == 0) {
+                e = i;                                   // w_N^i
+            } else {
+                long long rr = i / g.ns, kk = i % g.ns;  // entry r * ns + k
+                e = kk * rr;
+            }
+            double sn, cs;
+            sincospi(-2.0 * (double)(e % g.N) / (double)g.N, &sn, &cs);
+            base[g.offset + i] = make_float2((float)cs, (float)sn);
+            return;
+        }
+        i -= g.count;
+    }
+}
+
+cudaError_t launch_make_tables(float2 *base, const TableSegs &segs, cudaStream_t s) {
+    long long total = 0;
+    for (int i = 0; i < segs.n; i++) total += segs.seg[i].count;
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    spectre_make_tables<<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(base, segs);
+    return cudaGetLastError();
 }
 
 cudaError_t upload_w64(const float2 *host64) {

@@ -117,4 +117,24 @@ void slice_geometry(int M, int *threads_per_slice, int *slices_per_block, size_t
 // Upload exp(-2 pi i e / 64), e < 64, to the constant bank of the current device.
 cudaError_t upload_w64(const float2 *host64);
 
+// Fixed scratch of the no-allocation entry point (kernels.cu).
+constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;
+// Device address of the scratch on the current device.  The first call on a
+// device looks it up (and loads the constant twiddles); later calls reuse it.
+cudaError_t noalloc_scratch(void **ptr);
+
+// One segment of twiddle table: count entries at base + offset.  ns == 0:
+// entry i = w_N^i.  ns > 0: entry r * ns + k = w_N^{k r} (a slice-pass table).
+struct TableSeg {
+    long long offset;
+    long long count;
+    long long ns;
+    long long N;
+};
+struct TableSegs {
+    int n;
+    TableSeg seg[1 + 2 * kMaxPasses];
+};
+cudaError_t launch_make_tables(float2 *base, const TableSegs &segs, cudaStream_t s);
+
 }  // namespace spectre
