@@ -258,7 +258,10 @@ def native_arm(args, w, rank, world, local_rank):
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.05)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    R, M, nf, wave_ch, nlaunch = mix.plan
+    nwaves = (nlaunch - 1) // 2
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nlaunch + 1)]
+              for _ in range(args.steps)]
     for ev in events:  # torch creates the CUDA event on its first record
         for e in ev:
             e.record(stream)
@@ -276,8 +279,14 @@ def native_arm(args, w, rank, world, local_rank):
     sampler.stop()
     clocks = sampler.summary(t_host0, t_host1)
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in events]
-    kern_ms = [[e[j].elapsed_time(e[j + 1]) for e in events] for j in range(3)]
+    step_ms = [e[0].elapsed_time(e[-1]) for e in events]
+    # launch i of a step: row pass of wave i//2 (even i < 2 waves), slice pass
+    # (odd i), inverse row pass (last); per-kernel time = sum over its launches
+    kern_ms = [[0.0] * args.steps for _ in range(3)]
+    for s_i, e in enumerate(events):
+        for i in range(nlaunch):
+            kind = 2 if i == nlaunch - 1 else (i % 2)
+            kern_ms[kind][s_i] += e[i].elapsed_time(e[i + 1])
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -324,7 +333,8 @@ def native_arm(args, w, rank, world, local_rank):
     kmean = [sum(k) / len(k) for k in kern_ms]
     ksum = sum(kmean)
     kernels = [{"name": n, "ms": round(m, 5), "share": round(m / ksum, 4),
-                "dram_bytes": per_kernel_traffic.get(n)} for n, m in zip(names, kmean)]
+                "launches_per_step": (nwaves if i < 2 else 1),
+                "dram_bytes": per_kernel_traffic.get(n)} for i, (n, m) in enumerate(zip(names, kmean))]
     dom = max(range(3), key=lambda i: kmean[i])
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -335,6 +345,8 @@ def native_arm(args, w, rank, world, local_rank):
                  "G[:, :F] + gamma, beta read + y written",
         "algorithmic_bytes": alg_bytes, "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
         "kernels": kernels, "dominant_kernel": names[dom],
+        "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
+                 "launches_per_step": nlaunch},
     }
 
     # ---- CPU baseline (rank 0, N = 1 only)
@@ -363,7 +375,7 @@ def native_arm(args, w, rank, world, local_rank):
             "config": config_dict(w, world),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": nlaunch * args.steps,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "clocks": clocks,

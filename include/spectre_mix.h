@@ -117,17 +117,18 @@ int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k,
                          void *stream);
 
 /*
- * As spectre_mix_run, and also records the CUDA events events[0..3] on
- * `stream` around the three kernel launches of the path: events[0] before
- * the row pass, events[1] before the slice pass, events[2] before the
- * inverse row pass, events[3] after it.  `events` points to 4 cudaEvent_t
- * created by the caller.  For per-kernel timing; the launches are the same
- * as spectre_mix_run's.
+ * As spectre_mix_run, and also records CUDA events on `stream` around every
+ * kernel launch of the path, for per-kernel timing.  The path is, for each
+ * channel wave w (see spectre_mix_plan_info), a row-pass launch then a
+ * slice-pass launch, and finally one inverse-row-pass launch: n launches in
+ * all.  `events` points to nevents = n + 1 cudaEvent_t created by the caller;
+ * events[i] is recorded before launch i and events[n] after the last.
+ * Returns SPECTRE_ERR_ARG if nevents != n + 1 or an event is NULL.
  */
 int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k,
                              const void *v, const void *x, const float *G,
                              const float *gamma, const float *beta, void *y,
-                             void *const *events, void *stream);
+                             void *const *events, int nevents, void *stream);
 
 /*
  * One mix that allocates nothing.  The pages have no counterpart: this entry
@@ -147,8 +148,9 @@ int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k,
  * over from the previous call.
  *
  *   Returns SPECTRE_ERR_SCRATCH when the tables plus the workspace of this
- *   shape (4 * B * C * (R/2+1) * M * 8 bytes, see spectre_mix_plan_info)
- *   exceed the scratch; other errors as spectre_mix_create/spectre_mix_run.
+ *   shape (what spectre_mix_workspace_bytes reports for the same shape's
+ *   plan, without staging) exceed the scratch; other errors as
+ *   spectre_mix_create/spectre_mix_run.
  *
  * The first call on a device looks up the scratch's device address and loads
  * constant twiddles (synchronous); make that first call before any stream
@@ -169,15 +171,19 @@ int spectre_mix_destroy(spectre_mix_t h);
 /* Static, human-readable text for a status code. */
 const char *spectre_mix_error_string(int code);
 
-/* Device bytes held by the handle (tables + workspace), 0 for NULL. */
+/* Device bytes held by the handle (tables, workspace, staging), 0 for NULL. */
 size_t spectre_mix_workspace_bytes(spectre_mix_t h);
 
 /*
  * The decomposition the plan chose: L = R * M, with R-point transforms in the
- * row passes and M-point transforms per frequency slice.  Any out-pointer may
- * be NULL.  Returns SPECTRE_ERR_ARG for a NULL handle.
+ * row passes and M-point transforms per frequency slice (R/2 + 1 slices per
+ * channel).  Channels are processed in waves of `channels_per_wave` so that
+ * one wave's row-pass output stays in L2 until the slice pass reads it;
+ * `launches` is the number of kernel launches of one run (2 per wave + 1).
+ * Any out-pointer may be NULL.  Returns SPECTRE_ERR_ARG for a NULL handle.
  */
-int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_channel);
+int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_channel,
+                          int *channels_per_wave, int *launches);
 
 #ifdef __cplusplus
 }

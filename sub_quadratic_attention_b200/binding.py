@@ -36,12 +36,12 @@ SIGNATURES = {
     "spectre_mix_run": (_i, [_vp] * 10),
     "spectre_mix_run_debug": (_i, [_vp] * 11),
     "spectre_mix_run_host": (_i, [_vp] * 10),
-    "spectre_mix_run_profiled": (_i, [_vp] * 11),
+    "spectre_mix_run_profiled": (_i, [_vp] * 10 + [_i, _vp]),
     "spectre_mix_run_noalloc": (_i, [_i] * 6 + [ctypes.c_float] + [_vp] * 9),
     "spectre_mix_destroy": (_i, [_vp]),
     "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
     "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
-    "spectre_mix_plan_info": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "spectre_mix_plan_info": (_i, [_vp] + [ctypes.POINTER(_i)] * 5),
 }
 
 
@@ -133,12 +133,12 @@ def spectre_mix_run_host(h: int, q, k, v, x, G, gamma, beta, y, stream=None) -> 
 
 
 def spectre_mix_run_profiled(h: int, q, k, v, x, G, gamma, beta, y, events, stream=None) -> None:
-    """``events``: four ``torch.cuda.Event(enable_timing=True)`` recorded around
-    the three kernel launches."""
-    arr = (_vp * 4)(*[e.cuda_event for e in events])
+    """``events``: launches + 1 ``torch.cuda.Event(enable_timing=True)`` (already
+    created), recorded before every kernel launch and after the last."""
+    arr = (_vp * len(events))(*[e.cuda_event for e in events])
     _check(_lib.spectre_mix_run_profiled(h, _ptr(q), _ptr(k), _ptr(v), _ptr(x), _ptr(G),
                                          _ptr(gamma), _ptr(beta), _ptr(y),
-                                         ctypes.cast(arr, _vp), _stream(stream)),
+                                         ctypes.cast(arr, _vp), len(events), _stream(stream)),
            "spectre_mix_run_profiled")
 
 
@@ -165,11 +165,11 @@ def spectre_mix_workspace_bytes(h: Optional[int]) -> int:
     return int(_lib.spectre_mix_workspace_bytes(h))
 
 
-def spectre_mix_plan_info(h: int) -> Tuple[int, int, int]:
-    R, M, S = _i(), _i(), _i()
-    _check(_lib.spectre_mix_plan_info(h, ctypes.byref(R), ctypes.byref(M), ctypes.byref(S)),
-           "spectre_mix_plan_info")
-    return R.value, M.value, S.value
+def spectre_mix_plan_info(h: int) -> Tuple[int, int, int, int, int]:
+    """(R, M, slices per channel, channels per wave, kernel launches per run)."""
+    vals = [_i() for _ in range(5)]
+    _check(_lib.spectre_mix_plan_info(h, *[ctypes.byref(v) for v in vals]), "spectre_mix_plan_info")
+    return tuple(v.value for v in vals)
 
 
 class SpectreMix:
@@ -208,7 +208,7 @@ class SpectreMix:
         return spectre_mix_workspace_bytes(self.handle)
 
     @property
-    def plan(self) -> Tuple[int, int, int]:
+    def plan(self) -> Tuple[int, int, int, int, int]:
         return spectre_mix_plan_info(self.handle)
 
     def close(self) -> None:

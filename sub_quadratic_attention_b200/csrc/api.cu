@@ -15,20 +15,35 @@
 
 using namespace spectre;
 
-struct spectre_mix_s {
-    int device;
+// Shape, decomposition and launch geometry of one problem.
+struct PathGeom {
     int B, L, H, D, C, F, dtype;
     float eps;
     int R, M, NF;
-    // device memory owned by the handle
-    void *tables;       // twL followed by the slice tables
-    float2 *twL;
-    SliceTables tabs;
-    float2 *A, *P;
-    size_t table_bytes, ws_bytes;
-    // geometry
+    int W;               // channels per wave (A of one wave kept in L2)
+    int p16;             // P stored as fp16 with per-slice scales (bf16 I/O)
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
+    size_t a_bytes, p_bytes, s_bytes;
+};
+
+// Device buffers the launch sequence works in.
+struct PathBuffers {
+    const float2 *twL;
+    SliceTables tabs;
+    float2 *A;           // [3][B][W][NF][M]
+    void *P;             // [B][C][NF][M] float2 or __half2
+    float *pscale;       // [B][C][NF]
+};
+
+struct spectre_mix_s {
+    int device;
+    PathGeom g;
+    // device memory owned by the handle
+    void *tables;       // twL followed by the slice tables
+    void *ws;           // A, P, pscale
+    PathBuffers bufs;
+    size_t table_bytes, ws_bytes;
     // staging for spectre_mix_run_host, allocated on first use
     void *stage;
     size_t stage_bytes;
@@ -97,10 +112,127 @@ int check_device(int *dev_out) {
 void free_handle(spectre_mix_s *h) {
     if (!h) return;
     if (h->tables) cudaFree(h->tables);
-    if (h->A) cudaFree(h->A);
-    if (h->P) cudaFree(h->P);
+    if (h->ws) cudaFree(h->ws);
     if (h->stage) cudaFree(h->stage);
     delete h;
+}
+
+// Validate a shape and derive its geometry.  l2_bytes sizes the channel
+// waves: one wave's A (3 signals x B x W channels x (R/2+1) x M complex fp32)
+// is kept within half of L2 so the slice pass reads it back from L2.
+int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2_bytes, PathGeom *g) {
+    if (B < 1 || B > 65535 || H < 1 || D < 1 || L < 1) return SPECTRE_ERR_ARG;
+    if (dtype != SPECTRE_F32 && dtype != SPECTRE_BF16) return SPECTRE_ERR_ARG;
+    if (!(eps > 0.0f) || !std::isfinite(eps)) return SPECTRE_ERR_ARG;
+    if ((long long)H * D > (1 << 20)) return SPECTRE_ERR_ARG;
+    int R = 0, M = 0;
+    if (!choose_split(L, &R, &M)) return SPECTRE_ERR_UNSUPPORTED_L;
+    if (F < 1 || F > L / 2 + 1) return SPECTRE_ERR_ARG;
+    const int C = H * D;
+    const int NF = R / 2 + 1;
+    // inverse row pass: R rows x T2C x padded C floats must fit one block's smem
+    const int ZS = (int)align_up((size_t)C, 32) + 16;
+    if ((size_t)R * ZS * sizeof(float) > 227 * 1024) return SPECTRE_ERR_ARG;
+    g->B = B; g->L = L; g->H = H; g->D = D; g->C = C; g->F = F; g->dtype = dtype; g->eps = eps;
+    g->R = R; g->M = M; g->NF = NF;
+    g->ZS = ZS;
+    g->p16 = dtype == SPECTRE_BF16 ? 1 : 0;
+    // channel waves: with kWaveL2Fraction > 0, one wave's A is sized to that
+    // fraction of L2 so the slice pass could read it back from L2.  Measured on
+    // B200 for the bf16 long workload, waves were slower (each wave's grid
+    // fills the SMs only ~1.2 times and L2 still wrote most of A back to
+    // DRAM), so the plan uses a single wave.
+    constexpr double kWaveL2Fraction = 0.0;
+    const size_t per_ch = (size_t)3 * B * NF * M * sizeof(float2);
+    const size_t budget = (size_t)(kWaveL2Fraction * (double)l2_bytes);
+    int W = C;
+    if (budget > 0 && per_ch * (size_t)C > budget) {
+        size_t w = budget / per_ch;
+        w -= w % 64;
+        if (w >= 64) W = (int)w;
+    }
+    g->W = W;
+    // inverse row pass: register-resident LayerNorm when a block of
+    // T2C x ceil(C/2) <= 1024 threads covers the channels; else the
+    // shared-memory variant (R rows x T2C x padded C floats per block)
+    const int CP = (C + 1) / 2;
+    g->inv_reg = (R <= 16 && CP <= 1024) ? 1 : 0;
+    int T2C;
+    if (g->inv_reg) {
+        T2C = 1;
+        while (T2C < 8 && T2C * 2 * CP <= (CP > 512 ? 1024 : 512) && T2C * 2 <= M) T2C *= 2;
+    } else {
+        T2C = 8;
+        while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
+    }
+    g->T2C = T2C;
+    const size_t slices = (size_t)B * C * NF;
+    g->a_bytes = align_up((size_t)3 * B * W * NF * M * sizeof(float2), 256);
+    g->p_bytes = align_up(slices * M * (g->p16 ? 4 : 8), 256);
+    g->s_bytes = align_up(slices * sizeof(float), 256);
+    return SPECTRE_OK;
+}
+
+int wave_count(const PathGeom &g) { return (g.C + g.W - 1) / g.W; }
+
+// The launch sequence of one mix: per channel wave the row pass then the
+// slice pass, then the inverse row pass with residual + LayerNorm.  events
+// (nullable, 2 * waves + 2 of them) are recorded before every launch and
+// after the last.
+int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const void *k, const void *v,
+                const void *x, const float *G, const float *gamma, const float *beta, void *y,
+                float *out_f32, void *const *events, cudaStream_t s) {
+    int ev = 0;
+    auto mark = [&]() -> cudaError_t {
+        return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s) : cudaSuccess;
+    };
+    cudaError_t e = cudaSuccess;
+    for (int c_lo = 0; c_lo < g.C; c_lo += g.W) {
+        const int Cw = g.C - c_lo < g.W ? g.C - c_lo : g.W;
+        RowsFwdArgs fa;
+        fa.q = q; fa.k = k; fa.v = v;
+        fa.A = bf.A;
+        fa.twL = bf.twL;
+        fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
+        fa.c_lo = c_lo; fa.Cw = Cw;
+        fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
+        e = mark();
+        if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, s);
+        if (e != cudaSuccess) return cuda_status(e);
+
+        SliceArgs sa;
+        sa.A = bf.A; sa.P = bf.P; sa.pscale = bf.pscale; sa.twL = bf.twL; sa.G = G; sa.tabs = bf.tabs;
+        sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
+        sa.c_lo = c_lo; sa.Cw = Cw;
+        sa.p16 = g.p16;
+        sa.nbins = g.L / 2 + 1;
+        sa.nslices = (long long)g.B * Cw * g.NF;
+        sa.invL = 1.0f / (float)g.L;
+        e = mark();
+        if (e == cudaSuccess) e = launch_slices(sa, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    RowsInvArgs ia;
+    ia.P = bf.P; ia.pscale = bf.pscale;
+    ia.x = x; ia.gamma = gamma; ia.beta = beta; ia.y = y; ia.out_f32 = out_f32;
+    ia.B = g.B; ia.L = g.L; ia.M = g.M; ia.C = g.C;
+    ia.T2C = g.T2C; ia.ZS = g.ZS; ia.eps = g.eps;
+    ia.reg_variant = g.inv_reg;
+    ia.vec2 = (g.C % 2 == 0) ? 1 : 0;
+    e = mark();
+    if (e == cudaSuccess) e = launch_rows_inv_ln(g.R, g.dtype, ia, s);
+    if (e == cudaSuccess) e = mark();
+    if (e != cudaSuccess) return cuda_status(e);
+    return SPECTRE_OK;
+}
+
+size_t l2_size(int dev) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess || v <= 0) {
+        cudaGetLastError();
+        return (size_t)32 << 20;
+    }
+    return (size_t)v;
 }
 
 }  // namespace
@@ -124,47 +256,22 @@ const char *spectre_mix_error_string(int code) {
 int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, int dtype, float eps) {
     if (!out) return SPECTRE_ERR_ARG;
     *out = nullptr;
-    if (B < 1 || B > 65535 || H < 1 || D < 1 || L < 1) return SPECTRE_ERR_ARG;
-    if (dtype != SPECTRE_F32 && dtype != SPECTRE_BF16) return SPECTRE_ERR_ARG;
-    if (!(eps > 0.0f) || !std::isfinite(eps)) return SPECTRE_ERR_ARG;
-    if ((long long)H * D > (1 << 20)) return SPECTRE_ERR_ARG;
-    int R = 0, M = 0;
-    if (!choose_split(L, &R, &M)) return SPECTRE_ERR_UNSUPPORTED_L;
-    if (F < 1 || F > L / 2 + 1) return SPECTRE_ERR_ARG;
-    const int C = H * D;
-    const int NF = R / 2 + 1;
-    // inverse row pass: R rows x T2C x padded C floats must fit one block's smem
-    const int ZS = (int)align_up((size_t)C, 32) + 16;
-    const size_t smem_max = 227 * 1024;
-    if ((size_t)R * ZS * sizeof(float) > smem_max) return SPECTRE_ERR_ARG;
+    PathGeom g;
+    // validate with a provisional L2 size; the waves are re-derived below
+    int st = make_geom(B, L, H, D, F, dtype, eps, (size_t)32 << 20, &g);
+    if (st != SPECTRE_OK) return st;
     if (fault_requested("alloc")) return SPECTRE_ERR_NOMEM;
 
     int dev = -1;
-    int st = check_device(&dev);
+    st = check_device(&dev);
     if (st != SPECTRE_OK) return st;
+    make_geom(B, L, H, D, F, dtype, eps, l2_size(dev), &g);
 
     spectre_mix_s *h = new (std::nothrow) spectre_mix_s();
     if (!h) return SPECTRE_ERR_NOMEM;
     h->device = dev;
-    h->B = B; h->L = L; h->H = H; h->D = D; h->C = C; h->F = F; h->dtype = dtype; h->eps = eps;
-    h->R = R; h->M = M; h->NF = NF;
-
-    // ---- geometry
-    // inverse row pass: register-resident LayerNorm when a block of
-    // T2C x ceil(C/2) <= 1024 threads covers the channels; else the
-    // shared-memory variant (R rows x T2C x padded C floats per block)
-    const int CP = (C + 1) / 2;
-    h->inv_reg = (R <= 16 && CP <= 1024) ? 1 : 0;
-    int T2C;
-    if (h->inv_reg) {
-        T2C = 1;
-        while (T2C < 8 && T2C * 2 * CP <= (CP > 512 ? 1024 : 512) && T2C * 2 <= M) T2C *= 2;
-    } else {
-        T2C = 8;
-        while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
-    }
-    h->T2C = T2C;
-    h->ZS = ZS;
+    h->g = g;
+    const int M = g.M;
 
     // ---- twiddle tables (double on the host, stored fp32)
     const RadList sch = make_schedule(M);
@@ -210,21 +317,23 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
         free_handle(h);
         return cuda_status(e);
     }
-    h->twL = static_cast<float2 *>(h->tables);
+    h->bufs.twL = static_cast<float2 *>(h->tables);
     for (int d = 0; d < 2; d++)
         for (int p = 0; p < kMaxPasses; p++)
-            h->tabs.tw[d][p] = (p > 0 && p < sch.n) ? h->twL + offs[d][p] : nullptr;
+            h->bufs.tabs.tw[d][p] = (p > 0 && p < sch.n) ? h->bufs.twL + offs[d][p] : nullptr;
 
-    // ---- workspace
-    const size_t slice_elems = (size_t)B * C * NF * M;
-    e = cudaMalloc(reinterpret_cast<void **>(&h->A), 3 * slice_elems * sizeof(float2));
-    if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void **>(&h->P), slice_elems * sizeof(float2));
+    // ---- workspace: A of one wave, P, P scales
+    h->ws_bytes = g.a_bytes + g.p_bytes + g.s_bytes;
+    e = cudaMalloc(&h->ws, h->ws_bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
         free_handle(h);
         return cuda_status(e);
     }
-    h->ws_bytes = 4 * slice_elems * sizeof(float2);
+    char *base = static_cast<char *>(h->ws);
+    h->bufs.A = reinterpret_cast<float2 *>(base);
+    h->bufs.P = base + g.a_bytes;
+    h->bufs.pscale = reinterpret_cast<float *>(base + g.a_bytes + g.p_bytes);
     *out = h;
     return SPECTRE_OK;
 }
@@ -243,42 +352,8 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
         return SPECTRE_ERR_DEVICE;
     }
     if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    auto mark = [&](int i) -> cudaError_t {
-        return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s) : cudaSuccess;
-    };
-
-    RowsFwdArgs fa;
-    fa.q = q; fa.k = k; fa.v = v;
-    fa.A = h->A;
-    fa.twL = h->twL;
-    fa.B = h->B; fa.L = h->L; fa.M = h->M; fa.C = h->C;
-    fa.vec2 = (h->C % 2 == 0) ? 1 : 0;
-    cudaError_t e = mark(0);
-    if (e == cudaSuccess) e = launch_rows_fwd(h->R, h->dtype, fa, s);
-    if (e != cudaSuccess) return cuda_status(e);
-
-    SliceArgs sa;
-    sa.A = h->A; sa.P = h->P; sa.twL = h->twL; sa.G = G; sa.tabs = h->tabs;
-    sa.B = h->B; sa.L = h->L; sa.R = h->R; sa.M = h->M; sa.C = h->C; sa.D = h->D; sa.F = h->F;
-    sa.nbins = h->L / 2 + 1;
-    sa.nslices = (long long)h->B * h->C * h->NF;
-    sa.invL = 1.0f / (float)h->L;
-    e = mark(1);
-    if (e == cudaSuccess) e = launch_slices(sa, s);
-    if (e != cudaSuccess) return cuda_status(e);
-
-    RowsInvArgs ia;
-    ia.P = h->P; ia.x = x; ia.gamma = gamma; ia.beta = beta; ia.y = y; ia.out_f32 = out_f32;
-    ia.B = h->B; ia.L = h->L; ia.M = h->M; ia.C = h->C;
-    ia.T2C = h->T2C; ia.ZS = h->ZS; ia.eps = h->eps;
-    ia.reg_variant = h->inv_reg;
-    ia.vec2 = (h->C % 2 == 0) ? 1 : 0;
-    e = mark(2);
-    if (e == cudaSuccess) e = launch_rows_inv_ln(h->R, h->dtype, ia, s);
-    if (e == cudaSuccess) e = mark(3);
-    if (e != cudaSuccess) return cuda_status(e);
-    return SPECTRE_OK;
+    return launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, out_f32, events,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int spectre_mix_run(spectre_mix_t h, const void *q, const void *k, const void *v, const void *x,
@@ -294,8 +369,12 @@ int spectre_mix_run_debug(spectre_mix_t h, const void *q, const void *k, const v
 
 int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k, const void *v,
                              const void *x, const float *G, const float *gamma, const float *beta,
-                             void *y, void *const *events, void *stream) {
-    if (!events || !events[0] || !events[1] || !events[2] || !events[3]) return SPECTRE_ERR_ARG;
+                             void *y, void *const *events, int nevents, void *stream) {
+    if (!h || !events) return SPECTRE_ERR_ARG;
+    const int need = 2 * wave_count(h->g) + 2;
+    if (nevents != need) return SPECTRE_ERR_ARG;
+    for (int i = 0; i < need; i++)
+        if (!events[i]) return SPECTRE_ERR_ARG;
     return run_impl(h, q, k, v, x, G, gamma, beta, y, nullptr, events, stream);
 }
 
@@ -308,10 +387,11 @@ int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k, const vo
         cudaGetLastError();
         return SPECTRE_ERR_DEVICE;
     }
-    const size_t es = h->dtype == SPECTRE_F32 ? 4 : 2;
-    const size_t nt = (size_t)h->B * h->L * h->C * es;
-    const size_t ng = (size_t)h->H * (h->L / 2 + 1) * sizeof(float);
-    const size_t nc = (size_t)h->C * sizeof(float);
+    const PathGeom &g = h->g;
+    const size_t es = g.dtype == SPECTRE_F32 ? 4 : 2;
+    const size_t nt = (size_t)g.B * g.L * g.C * es;
+    const size_t ng = (size_t)g.H * (g.L / 2 + 1) * sizeof(float);
+    const size_t nc = (size_t)g.C * sizeof(float);
     const size_t o_t = align_up(nt, 256), o_g = align_up(ng, 256), o_c = align_up(nc, 256);
     const size_t need = 5 * o_t + o_g + 2 * o_c;
     if (!h->stage) {
@@ -354,25 +434,21 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
                             const void *k, const void *v, const void *x, const float *G,
                             const float *gamma, const float *beta, void *y, void *stream) {
     // the same validation as spectre_mix_create and spectre_mix_run
-    if (B < 1 || B > 65535 || H < 1 || D < 1 || L < 1) return SPECTRE_ERR_ARG;
-    if (dtype != SPECTRE_F32 && dtype != SPECTRE_BF16) return SPECTRE_ERR_ARG;
-    if (!(eps > 0.0f) || !std::isfinite(eps)) return SPECTRE_ERR_ARG;
-    if ((long long)H * D > (1 << 20)) return SPECTRE_ERR_ARG;
-    int R = 0, M = 0;
-    if (!choose_split(L, &R, &M)) return SPECTRE_ERR_UNSUPPORTED_L;
-    if (F < 1 || F > L / 2 + 1) return SPECTRE_ERR_ARG;
-    const int C = H * D;
-    const int NF = R / 2 + 1;
-    const int ZS = (int)align_up((size_t)C, 32) + 16;
-    if ((size_t)R * ZS * sizeof(float) > 227 * 1024) return SPECTRE_ERR_ARG;
+    PathGeom g;
+    int st = make_geom(B, L, H, D, F, dtype, eps, (size_t)32 << 20, &g);
+    if (st != SPECTRE_OK) return st;
     if (!q || !k || !v || !x || !G || !gamma || !beta || !y) return SPECTRE_ERR_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(x) || !aligned16(G) ||
         !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
         return SPECTRE_ERR_ALIGN;
+    int dev = -1;
+    st = check_device(&dev);
+    if (st != SPECTRE_OK) return st;
+    make_geom(B, L, H, D, F, dtype, eps, l2_size(dev), &g);
 
     // scratch layout: twiddle tables (as spectre_mix_create lays them out),
-    // then A [3][B][C][NF][M] and P [B][C][NF][M], all fp32 complex
-    const RadList sch = make_schedule(M);
+    // then A of one wave, P and the P scales
+    const RadList sch = make_schedule(g.M);
     TableSegs segs;
     segs.n = 0;
     size_t n_tab = (size_t)L / 2 + 1;
@@ -391,13 +467,8 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
         }
     }
     const size_t tab_bytes = align_up(n_tab * sizeof(float2), 256);
-    const size_t slice_elems = (size_t)B * C * NF * M;
-    const size_t need = tab_bytes + 4 * slice_elems * sizeof(float2);
+    const size_t need = tab_bytes + g.a_bytes + g.p_bytes + g.s_bytes;
     if (need > kNoAllocScratchBytes) return SPECTRE_ERR_SCRATCH;
-
-    int dev = -1;
-    int st = check_device(&dev);
-    if (st != SPECTRE_OK) return st;
     if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
     void *scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
@@ -406,55 +477,22 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
         return cuda_status(e);
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float2 *tw = static_cast<float2 *>(scratch);
-    float2 *A = reinterpret_cast<float2 *>(static_cast<char *>(scratch) + tab_bytes);
-    float2 *P = A + 3 * slice_elems;
-    e = launch_make_tables(tw, segs, s);
-    if (e != cudaSuccess) return cuda_status(e);
-
-    SliceTables tabs;
+    char *base = static_cast<char *>(scratch);
+    PathBuffers bf;
+    float2 *tw = reinterpret_cast<float2 *>(base);
+    bf.twL = tw;
+    bf.A = reinterpret_cast<float2 *>(base + tab_bytes);
+    bf.P = base + tab_bytes + g.a_bytes;
+    bf.pscale = reinterpret_cast<float *>(base + tab_bytes + g.a_bytes + g.p_bytes);
     {
         int si = 1;
         for (int d = 0; d < 2; d++)
             for (int p = 0; p < kMaxPasses; p++)
-                tabs.tw[d][p] = (p > 0 && p < sch.n) ? tw + segs.seg[si++].offset : nullptr;
+                bf.tabs.tw[d][p] = (p > 0 && p < sch.n) ? tw + segs.seg[si++].offset : nullptr;
     }
-    const int CP = (C + 1) / 2;
-    const int inv_reg = (R <= 16 && CP <= 1024) ? 1 : 0;
-    int T2C;
-    if (inv_reg) {
-        T2C = 1;
-        while (T2C < 8 && T2C * 2 * CP <= (CP > 512 ? 1024 : 512) && T2C * 2 <= M) T2C *= 2;
-    } else {
-        T2C = 8;
-        while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
-    }
-
-    RowsFwdArgs fa;
-    fa.q = q; fa.k = k; fa.v = v; fa.A = A; fa.twL = tw;
-    fa.B = B; fa.L = L; fa.M = M; fa.C = C;
-    fa.vec2 = (C % 2 == 0) ? 1 : 0;
-    e = launch_rows_fwd(R, dtype, fa, s);
+    e = launch_make_tables(tw, segs, s);
     if (e != cudaSuccess) return cuda_status(e);
-
-    SliceArgs sa;
-    sa.A = A; sa.P = P; sa.twL = tw; sa.G = G; sa.tabs = tabs;
-    sa.B = B; sa.L = L; sa.R = R; sa.M = M; sa.C = C; sa.D = D; sa.F = F;
-    sa.nbins = L / 2 + 1;
-    sa.nslices = (long long)B * C * NF;
-    sa.invL = 1.0f / (float)L;
-    e = launch_slices(sa, s);
-    if (e != cudaSuccess) return cuda_status(e);
-
-    RowsInvArgs ia;
-    ia.P = P; ia.x = x; ia.gamma = gamma; ia.beta = beta; ia.y = y; ia.out_f32 = nullptr;
-    ia.B = B; ia.L = L; ia.M = M; ia.C = C;
-    ia.T2C = T2C; ia.ZS = ZS; ia.eps = eps;
-    ia.reg_variant = inv_reg;
-    ia.vec2 = (C % 2 == 0) ? 1 : 0;
-    e = launch_rows_inv_ln(R, dtype, ia, s);
-    if (e != cudaSuccess) return cuda_status(e);
-    return SPECTRE_OK;
+    return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s);
 }
 
 int spectre_mix_destroy(spectre_mix_t h) {
@@ -477,11 +515,14 @@ size_t spectre_mix_workspace_bytes(spectre_mix_t h) {
     return h->table_bytes + h->ws_bytes + h->stage_bytes;
 }
 
-int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_channel) {
+int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_channel,
+                          int *channels_per_wave, int *launches) {
     if (!h) return SPECTRE_ERR_ARG;
-    if (R) *R = h->R;
-    if (M) *M = h->M;
-    if (slices_per_channel) *slices_per_channel = h->NF;
+    if (R) *R = h->g.R;
+    if (M) *M = h->g.M;
+    if (slices_per_channel) *slices_per_channel = h->g.NF;
+    if (channels_per_wave) *channels_per_wave = h->g.W;
+    if (launches) *launches = 2 * wave_count(h->g) + 1;
     return SPECTRE_OK;
 }
 

@@ -10,8 +10,10 @@
 //
 // The index algebra is in kernels.cuh.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "fft_regs.cuh"
 #include "kernels.cuh"
@@ -67,12 +69,14 @@ __global__ void __launch_bounds__(256, R <= 16 ? 3 : 1) spectre_rows_fwd(RowsFwd
     const int t2 = blockIdx.x * 8 + (warp & 1) * 4 + (lane & 3);
     const int cp = blockIdx.y * 32 + (warp >> 1) * 8 + (lane >> 2);
     const int b = blockIdx.z;
-    const int c0 = 2 * cp;
-    const bool live = (t2 < a.M) && (c0 < a.C);
-    const bool has1 = live && (c0 + 1 < a.C);
+    const int cl = 2 * cp;                 // channel within the wave
+    const int c0 = a.c_lo + cl;
+    const int cend = min(a.C, a.c_lo + a.Cw);
+    const bool live = (t2 < a.M) && (c0 < cend);
+    const bool has1 = live && (c0 + 1 < cend);
     const size_t rowstride = (size_t)a.M * a.C;
-    const size_t plane = (size_t)a.B * a.C * NF * a.M;
-    float2 *dst0 = a.A + ((size_t)b * a.C + c0) * NF * a.M + t2;
+    const size_t plane = (size_t)a.B * a.Cw * NF * a.M;
+    float2 *dst0 = a.A + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
     float2 *dst1 = dst0 + (size_t)NF * a.M;
 
 #pragma unroll 1
@@ -236,30 +240,63 @@ __device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bo
     }
 }
 
+// Store of one slice of P.  With p16 the slice's values are scaled by a power
+// of two s chosen from the slice's largest magnitude m (m s < 2^14) and stored
+// as fp16 (round to nearest); pscale receives 1/s.  Otherwise fp32.  smax is
+// this slice's shared max word, zeroed at kernel start.
+struct PStore {
+    void *dst;        // slice base (float2 * or __half2 *)
+    float *pscale;    // this slice's scale slot
+    int *smax;
+    bool live, p16;
+};
+
+__device__ __forceinline__ float slice_scale(PStore &ps, float local_max) {
+    if (!ps.p16) return 1.0f;
+    atomicMax(ps.smax, __float_as_int(local_max));
+    __syncthreads();
+    const float m = __int_as_float(*ps.smax);
+    int e = 0;
+    if (m > 0.f) frexpf(m, &e);   // m < 2^e
+    const int sexp = max(-126, min(126, 14 - e));
+    return ldexpf(1.0f, sexp);
+}
+
+__device__ __forceinline__ void pstore(const PStore &ps, int t2, float2 v, float s) {
+    if (!ps.live) return;
+    if (ps.p16)
+        static_cast<__half2 *>(ps.dst)[t2] = __floats2half2_rn(v.x * s, v.y * s);
+    else
+        static_cast<float2 *>(ps.dst)[t2] = v;
+}
+
 // Inverse (unscaled) M-point transform of the values thread j holds at
 // positions j + r NT, via conj -> forward passes in reversed radix order ->
 // conj; writes P[t2] = w_L^{-f1 t2} * result[t2].
 template <int M>
 __device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL], float2 *buf,
-                                                    const SliceTables &tb, int j, bool live,
-                                                    float2 *__restrict__ dst, const float2 *__restrict__ twL,
-                                                    int f1) {
+                                                    const SliceTables &tb, int j, PStore &ps,
+                                                    const float2 *__restrict__ twL, int f1) {
     using Cfg = SliceCfg<M>;
     constexpr int NP = Cfg::NP, NT = Cfg::NT, RL = Cfg::RL;
 #pragma unroll
     for (int r = 0; r < RL; r++) o[r] = cconj(o[r]);
     if constexpr (NP == 0) {
-        if (live) dst[0] = cconj(o[0]);  // f1 * 0 = 0: no twiddle
+        float2 v = cconj(o[0]);  // f1 * 0 = 0: no twiddle
+        float s = slice_scale(ps, fmaxf(fabsf(v.x), fabsf(v.y)));
+        pstore(ps, 0, v, s);
     } else if constexpr (NP == 1) {
         Dft<RL>::run(o);
         // single butterfly (j = 0): output r at position r
-        if (live) {
+        float mx = 0.f;
 #pragma unroll
-            for (int r = 0; r < RL; r++) {
-                float2 w = __ldg(twL + f1 * r);
-                dst[r] = cconj(cmul(o[r], w));
-            }
+        for (int r = 0; r < RL; r++) {
+            o[r] = cconj(cmul(o[r], __ldg(twL + f1 * r)));
+            mx = fmaxf(mx, fmaxf(fabsf(o[r].x), fabsf(o[r].y)));
         }
+        float s = slice_scale(ps, mx);
+#pragma unroll
+        for (int r = 0; r < RL; r++) pstore(ps, r, o[r], s);
     } else {
         // first inverse pass: radix RL, Ns = 1, registers -> smem
         Dft<RL>::run(o);
@@ -273,26 +310,39 @@ __device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL]
         constexpr int NBF = M / R;
         constexpr int NB = (NBF + NT - 1) / NT;
         const float2 *tw = tb.tw[1][NP - 1];
+        float2 v[NB][R];
+        float mx = 0.f;
 #pragma unroll
         for (int i = 0; i < NB; i++) {
             int bf = j + i * NT;
             if (NBF % NT == 0 || bf < NBF) {
-                float2 v[R];
 #pragma unroll
-                for (int r = 0; r < R; r++) v[r] = buf[spad(bf + r * NBF)];
+                for (int r = 0; r < R; r++) v[i][r] = buf[spad(bf + r * NBF)];
 #pragma unroll
-                for (int r = 1; r < R; r++) v[r] = cmul(v[r], __ldg(tw + bf + r * NBF));
-                Dft<R>::run(v);
-                if (live) {
+                for (int r = 1; r < R; r++) v[i][r] = cmul(v[i][r], __ldg(tw + bf + r * NBF));
+                Dft<R>::run(v[i]);
 #pragma unroll
-                    for (int r = 0; r < R; r++) {
-                        int t2 = bf + r * NBF;
-                        float2 w = __ldg(twL + f1 * t2);
-                        dst[t2] = cconj(cmul(v[r], w));
-                    }
+                for (int r = 0; r < R; r++) {
+                    v[i][r] = cconj(cmul(v[i][r], __ldg(twL + f1 * (bf + r * NBF))));
+                    mx = fmaxf(mx, fmaxf(fabsf(v[i][r].x), fabsf(v[i][r].y)));
                 }
             }
         }
+        float s = slice_scale(ps, mx);
+#pragma unroll
+        for (int i = 0; i < NB; i++) {
+            int bf = j + i * NT;
+            if (NBF % NT == 0 || bf < NBF) {
+#pragma unroll
+                for (int r = 0; r < R; r++) pstore(ps, bf + r * NBF, v[i][r], s);
+            }
+        }
+    }
+    if (ps.p16 && ps.live && j == 0) {
+        int e = 0;
+        const float m = __int_as_float(*ps.smax);
+        if (m > 0.f) frexpf(m, &e);
+        *ps.pscale = ldexpf(1.0f, -max(-126, min(126, 14 - e)));
     }
 }
 
@@ -305,32 +355,45 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     const int j = threadIdx.x % NT;
     float2 *buf = reinterpret_cast<float2 *>(smem_f4) + sl * Cfg::BUF;
     float2 *sbuf = reinterpret_cast<float2 *>(smem_f4) + Cfg::SPB * Cfg::BUF + sl * M;
+    __shared__ int smax[Cfg::SPB];
+    if (j == 0) smax[sl] = 0;
     const long long sid = (long long)blockIdx.x * Cfg::SPB + sl;
     const bool live = sid < a.nslices;
     const int NF = a.R / 2 + 1;
     const long long sidc = live ? sid : 0;
     const int f1 = (int)(sidc % NF);
-    const long long bc = sidc / NF;             // b * C + c
-    const int c = (int)(bc % a.C);
+    const long long bcl = sidc / NF;            // b * Cw + (c - c_lo)
+    const int b = (int)(bcl / a.Cw);
+    const int c = a.c_lo + (int)(bcl % a.Cw);
     const int h = c / a.D;
-    const size_t sig_stride = (size_t)a.B * a.C * NF * M;
-    const float2 *srcA = a.A + (size_t)bc * NF * M + (size_t)f1 * M;
-    float2 *dstP = a.P + (size_t)bc * NF * M + (size_t)f1 * M;
+    const size_t sig_stride = (size_t)a.B * a.Cw * NF * M;
+    const float2 *srcA = a.A + (size_t)bcl * NF * M + (size_t)f1 * M;
+    const size_t pslice = ((size_t)b * a.C + c) * NF + f1;
+    PStore ps;
+    ps.dst = a.p16 ? static_cast<void *>(static_cast<__half2 *>(a.P) + pslice * M)
+                   : static_cast<void *>(static_cast<float2 *>(a.P) + pslice * M);
+    ps.pscale = a.pscale + pslice;
+    ps.smax = &smax[sl];
+    ps.live = live;
+    ps.p16 = a.p16 != 0;
     const float *Gh = a.G + (size_t)h * a.nbins;
+    __syncthreads();  // smax initialised
 
     float2 x[RL];
     float2 s[RL];
     // each thread owns bins f = f1 + R (j + r NT), r < RL, of the product;
-    // with kProdGlobal the slice's P row holds S until it is overwritten
+    // with kProdGlobal S is parked in this slice's q row of A, which nothing
+    // reads once the q transform has passed its first stage
+    float2 *park = const_cast<float2 *>(srcA);
     auto put = [&](int r, float2 v) {
         if constexpr (PROD == kProdSmem) sbuf[j + r * NT] = v;
         else if constexpr (PROD == kProdRegs) s[r] = v;
-        else { if (live) dstP[j + r * NT] = v; }
+        else { if (live) park[j + r * NT] = v; }
     };
     auto get = [&](int r) -> float2 {
         if constexpr (PROD == kProdSmem) return sbuf[j + r * NT];
         else if constexpr (PROD == kProdRegs) return s[r];
-        else return live ? dstP[j + r * NT] : make_float2(0.f, 0.f);
+        else return live ? park[j + r * NT] : make_float2(0.f, 0.f);
     };
 
     // q: S = Q * G' / L
@@ -352,7 +415,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     slice_forward<M>(srcA + 2 * sig_stride, live, buf, a.tabs, j, x);
 #pragma unroll
     for (int r = 0; r < RL; r++) x[r] = cmul(get(r), x[r]);
-    slice_inverse_store<M>(x, buf, a.tabs, j, live, dstP, a.twL, f1);
+    slice_inverse_store<M>(x, buf, a.tabs, j, ps, a.twL, f1);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,6 +424,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
 template <int R, typename T, bool DEBUG_OUT>
 __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
+    constexpr bool P16 = std::is_same<T, __nv_bfloat16>::value;  // bf16 I/O: fp16 P
     extern __shared__ float4 smem_f4[];
     float *zbuf = reinterpret_cast<float *>(smem_f4);  // [R * T2C][ZS]
     const int T2C = a.T2C, ZS = a.ZS;
@@ -374,21 +438,30 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
         if (t2 >= a.M) continue;
         const int c0 = 2 * cp;
         const bool has1 = c0 + 1 < a.C;
-        const float2 *pa = a.P + ((size_t)b * a.C + c0) * NF * a.M + t2;
-        const float2 *pb = pa + (size_t)NF * a.M;
+        const size_t sa = ((size_t)b * a.C + c0) * NF;
+        const size_t sb = sa + NF;
+        auto ld = [&](size_t slice, bool ok) -> float2 {
+            if (!ok) return make_float2(0.f, 0.f);
+            if constexpr (P16) {
+                float2 v = __half22float2(__ldg(static_cast<const __half2 *>(a.P) + slice * a.M + t2));
+                return cscale(v, __ldg(a.pscale + slice));
+            } else {
+                return __ldg(static_cast<const float2 *>(a.P) + slice * a.M + t2);
+            }
+        };
         float2 Z[R];
         {
-            float2 a0 = __ldg(pa), aN = __ldg(pa + (size_t)(R / 2) * a.M);
-            float2 b0 = has1 ? __ldg(pb) : make_float2(0.f, 0.f);
-            float2 bN = has1 ? __ldg(pb + (size_t)(R / 2) * a.M) : make_float2(0.f, 0.f);
+            float2 a0 = ld(sa, true), aN = ld(sa + R / 2, true);
+            float2 b0 = ld(sb, has1);
+            float2 bN = ld(sb + R / 2, has1);
             // DC and Nyquist: imaginary parts dropped; conj() for the inverse
             Z[0] = make_float2(a0.x, -b0.x);
             Z[R / 2] = make_float2(aN.x, -bN.x);
         }
 #pragma unroll
         for (int f1 = 1; f1 < R / 2; f1++) {
-            float2 pv = __ldg(pa + (size_t)f1 * a.M);
-            float2 qv = has1 ? __ldg(pb + (size_t)f1 * a.M) : make_float2(0.f, 0.f);
+            float2 pv = ld(sa + f1, true);
+            float2 qv = ld(sb + f1, has1);
             // Z[f1] = P_a + i P_b ; Z[R - f1] = conj(P_a) + i conj(P_b); stored conjugated
             Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
             Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
@@ -448,12 +521,39 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
 // shuffles and one shared-memory stage, in two passes (mean, then the mean
 // of squared deviations), in a fixed order.
 // ---------------------------------------------------------------------------
-template <int R, typename T, bool DEBUG_OUT>
+// Sum N per-lane values over the lanes that differ in lane bits [BIT, BITEND),
+// by recursive halving: at each bit a lane keeps half of its values and adds
+// the partner's copy of that half, so N values cost about N shuffles in all
+// rather than N per bit.  On return v[0 .. N >> (BITEND - BIT)) (at least one)
+// hold the sums of rows row0 + i.
+template <int N, int BIT, int BITEND> struct HalvingReduce {
+    __device__ __forceinline__ static void run(float *v, int lane, int &row0) {
+        if constexpr (BIT < BITEND && N > 1) {
+            constexpr int H = N / 2;
+            const bool up = (lane >> BIT) & 1;
+#pragma unroll
+            for (int i = 0; i < H; i++) {
+                const float keep = up ? v[i + H] : v[i];
+                const float send = up ? v[i] : v[i + H];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << BIT);
+            }
+            if (up) row0 += H;
+            HalvingReduce<H, BIT + 1, BITEND>::run(v, lane, row0);
+        } else if constexpr (BIT < BITEND) {
+#pragma unroll
+            for (int b = BIT; b < BITEND; b++) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1 << b);
+        }
+    }
+};
+
+constexpr int ilog2c(int v) { return v <= 1 ? 0 : 1 + ilog2c(v / 2); }
+
+template <int R, int T2C, typename T, bool DEBUG_OUT>
 __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
+    constexpr bool P16 = std::is_same<T, __nv_bfloat16>::value;  // bf16 I/O: fp16 P
     extern __shared__ float4 smem_f4[];
     float *part = reinterpret_cast<float *>(smem_f4);   // [nwarps][T2C][R], then stat[2][T2C][R]
-    const int T2C = a.T2C;
     const int nthr = blockDim.x;
     const int nwarps = nthr >> 5;
     float *stat = part + nwarps * T2C * R;               // [T2C][R]
@@ -467,17 +567,25 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     float z0[R], z1[R];
     {
         float2 Z[R];
-        const float2 *pa = a.P + ((size_t)b * a.C + c0) * NF * a.M + t2;
-        const float2 *pb = pa + (size_t)NF * a.M;
-        const float2 zero = make_float2(0.f, 0.f);
-        float2 a0 = live ? __ldg(pa) : zero, aN = live ? __ldg(pa + (size_t)(R / 2) * a.M) : zero;
-        float2 b0 = has1 ? __ldg(pb) : zero, bN = has1 ? __ldg(pb + (size_t)(R / 2) * a.M) : zero;
+        const size_t sa = ((size_t)b * a.C + c0) * NF;       // slice index of (c0, f1 = 0)
+        const size_t sb = sa + NF;
+        auto ld = [&](size_t slice, bool ok) -> float2 {
+            if (!ok) return make_float2(0.f, 0.f);
+            if constexpr (P16) {
+                float2 v = __half22float2(__ldg(static_cast<const __half2 *>(a.P) + slice * a.M + t2));
+                return cscale(v, __ldg(a.pscale + slice));
+            } else {
+                return __ldg(static_cast<const float2 *>(a.P) + slice * a.M + t2);
+            }
+        };
+        float2 a0 = ld(sa, live), aN = ld(sa + R / 2, live);
+        float2 b0 = ld(sb, has1), bN = ld(sb + R / 2, has1);
         Z[0] = make_float2(a0.x, -b0.x);
         Z[R / 2] = make_float2(aN.x, -bN.x);
 #pragma unroll
         for (int f1 = 1; f1 < R / 2; f1++) {
-            float2 pv = live ? __ldg(pa + (size_t)f1 * a.M) : zero;
-            float2 qv = has1 ? __ldg(pb + (size_t)f1 * a.M) : zero;
+            float2 pv = ld(sa + f1, live);
+            float2 qv = ld(sb + f1, has1);
             Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
             Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
         }
@@ -527,14 +635,18 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
                 s[t1] = live ? fmaf(d0, d0, has1 ? d1 * d1 : 0.f) : 0.f;
             }
         }
+        {
+            // channel pairs of one t2 differ in lane bits [log2 T2C, 5)
+            constexpr int B0 = ilog2c(T2C);
+            constexpr int NOUT = (R >> (5 - B0)) > 0 ? (R >> (5 - B0)) : 1;
+            float v[R];
 #pragma unroll
-        for (int t1 = 0; t1 < R; t1++)
-            for (int o = T2C; o < 32; o <<= 1) s[t1] += __shfl_xor_sync(0xffffffffu, s[t1], o);
-        if (lane < T2C) {
+            for (int t1 = 0; t1 < R; t1++) v[t1] = s[t1];
+            int row0 = 0;
+            HalvingReduce<R, B0, 5>::run(v, lane, row0);
 #pragma unroll
-            for (int t1 = 0; t1 < R; t1++) part[(warp * T2C + tl) * R + t1] = s[t1];
-        }
-        __syncthreads();
+            for (int i = 0; i < NOUT; i++) part[(warp * T2C + tl) * R + row0 + i] = v[i];
+        }        __syncthreads();
         for (int i = tid; i < T2C * R; i += nthr) {
             float acc = 0.f;
             for (int w = 0; w < nwarps; w++) acc += part[w * T2C * R + i];
@@ -566,7 +678,7 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
 // ---------------------------------------------------------------------------
 template <int R>
 static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a, cudaStream_t s) {
-    dim3 grid((a.M + 7) / 8, (a.C + 63) / 64, a.B);
+    dim3 grid((a.M + 7) / 8, (a.Cw + 63) / 64, a.B);
     if (dtype == 0)
         spectre_rows_fwd<R, float><<<grid, 256, 0, s>>>(a);
     else
@@ -644,10 +756,18 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
         const int CP = (a.C + 1) / 2;
         const int threads = ((a.T2C * CP + 31) / 32) * 32;
         size_t smem = (size_t)((threads / 32) * a.T2C * R + 2 * a.T2C * R) * sizeof(float);
-        if (a.out_f32)
-            spectre_rows_inv_ln_reg<R, T, true><<<grid, threads, smem, s>>>(a);
-        else
-            spectre_rows_inv_ln_reg<R, T, false><<<grid, threads, smem, s>>>(a);
+        switch (a.T2C) {
+#define SPECTRE_INV_T2C(t2c)                                                          \
+    case t2c:                                                                         \
+        if (a.out_f32)                                                                \
+            spectre_rows_inv_ln_reg<R, t2c, T, true><<<grid, threads, smem, s>>>(a);  \
+        else                                                                          \
+            spectre_rows_inv_ln_reg<R, t2c, T, false><<<grid, threads, smem, s>>>(a); \
+        break;
+            SPECTRE_INV_T2C(1) SPECTRE_INV_T2C(2) SPECTRE_INV_T2C(4) SPECTRE_INV_T2C(8)
+#undef SPECTRE_INV_T2C
+        default: return cudaErrorInvalidValue;
+        }
         return cudaGetLastError();
     }
     dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);

@@ -33,25 +33,30 @@ struct SliceTables {
 
 struct RowsFwdArgs {
     const void *q, *k, *v;
-    float2 *A;            // [3][B][C][R/2+1][M]
+    float2 *A;            // [3][B][Cw][R/2+1][M]: channels c_lo .. c_lo + Cw - 1
     const float2 *twL;    // exp(-2 pi i e / L), e in [0, L/2]
     int B, L, M, C;
+    int c_lo, Cw;         // channel wave (c_lo even)
     int vec2;             // C even: load channel pairs as one vector
 };
 
 struct SliceArgs {
-    const float2 *A;      // [3][B][C][R/2+1][M]
-    float2 *P;            // [B][C][R/2+1][M]
+    const float2 *A;      // [3][B][Cw][R/2+1][M]: the wave's channels
+    void *P;              // [B][C][R/2+1][M]: float2, or __half2 scaled by 1/pscale
+    float *pscale;        // [B][C][R/2+1]: P = stored * pscale (p16 only)
     const float2 *twL;
     const float *G;       // [H][L/2+1]
     SliceTables tabs;
     int B, L, R, M, C, D, F, nbins;
-    long long nslices;    // B * C * (R/2+1)
+    int c_lo, Cw;         // channel wave
+    int p16;              // store P as fp16 with a power-of-two scale per slice
+    long long nslices;    // B * Cw * (R/2+1)
     float invL;
 };
 
 struct RowsInvArgs {
-    const float2 *P;
+    const void *P;        // float2 (fp32 I/O) or __half2 (bf16 I/O) with pscale
+    const float *pscale;
     const void *x;
     const float *gamma, *beta;
     void *y;

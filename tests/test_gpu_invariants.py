@@ -5,6 +5,11 @@ L x L mixing matrix is circulant; §2.3: truncation keeps bins f < F).
 * a common circular shift of q and k leaves out unchanged;
 * a circular shift of v shifts out by the same amount;
 * out is linear in each of q, k, v (exactly, for a power-of-two scale);
+
+Shifted runs differ from the unshifted one by rounding only.  With bf16 I/O
+the slice-pass output P is stored in fp16 under a per-slice power-of-two
+scale: relative rounding error <= 2^-11 per value, about 4e-4 rms between two
+runs, so the shift checks allow 1e-3 there and 2e-5 for fp32 I/O (fp32 P).
 * q = k = v = cos(2 pi a t / L) gives out = (L^2 / 4) G[a] cos(2 pi a t / L)
   when a < F and 0 otherwise.
 """
@@ -41,11 +46,12 @@ def test_shift_and_scale_invariants(name):
     e["q"] = torch.roll(d["q"], s, 1)
     e["k"] = torch.roll(d["k"], s, 1)
     same = _out(w, e)
-    assert rel_l2(same.cpu().numpy(), base.double().cpu().numpy()) < 2e-5
+    tol = 1e-3 if w.dtype == "bf16" else 2e-5
+    assert rel_l2(same.cpu().numpy(), base.double().cpu().numpy()) < tol
     e = dict(d)
     e["v"] = torch.roll(d["v"], s, 1)
     shifted = _out(w, e)
-    assert rel_l2(shifted.cpu().numpy(), torch.roll(base, s, 1).double().cpu().numpy()) < 2e-5
+    assert rel_l2(shifted.cpu().numpy(), torch.roll(base, s, 1).double().cpu().numpy()) < tol
     for key in ("q", "k", "v"):
         e = dict(d)
         e[key] = d[key] * 2
