@@ -241,7 +241,8 @@ def native_arm(args, w, rank, world, local_rank):
     y = torch.empty_like(d["x"])
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps)
+    mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps,
+                             tensor_cores=args.tensor_cores)
     h = mix.handle
 
     def barrier():
@@ -346,7 +347,7 @@ def native_arm(args, w, rank, world, local_rank):
         "algorithmic_bytes": alg_bytes, "frac_of_8TBps_nominal": round(achieved / 8000.0, 4),
         "kernels": kernels, "dominant_kernel": names[dom],
         "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
-                 "launches_per_step": nlaunch},
+                 "launches_per_step": nlaunch, "tensor_core_dft16": bool(args.tensor_cores)},
     }
 
     # ---- CPU baseline (rank 0, N = 1 only)
@@ -394,6 +395,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tensor-cores", action="store_true",
+                    help="run the slice pass's DFT16 stages on tcgen05 (plan option)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -58,7 +58,8 @@ enum spectre_status {
     SPECTRE_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
     SPECTRE_ERR_NOMEM = -5,         /* device or host allocation failed */
     SPECTRE_ERR_DEVICE = -6,        /* no usable sm_100 device, or wrong current device */
-    SPECTRE_ERR_SCRATCH = -7        /* problem too large for the no-allocation scratch */
+    SPECTRE_ERR_SCRATCH = -7,       /* problem too large for the no-allocation scratch */
+    SPECTRE_ERR_TIMEOUT = -8        /* a bounded device-side wait gave up (see below) */
 };
 
 /* Size of the fixed device scratch behind spectre_mix_run_noalloc. */
@@ -163,6 +164,29 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype,
                             const void *v, const void *x, const float *G,
                             const float *gamma, const float *beta, void *y,
                             void *stream);
+
+enum spectre_option {
+    /* 0 (default): the slice pass's length-16 DFT stages run as CUDA-core
+     * butterflies.  1: they run on the tensor cores (tcgen05 MMA with fp16
+     * operands and fp32 accumulation against a DFT16/16 matrix), for bf16 I/O
+     * plans whose slice length M is 4096; other plans ignore the option.
+     * Measured on B200 for the bf16 long workload the tensor-core variant is
+     * slower (each stage waits for its MMA), hence the default. */
+    SPECTRE_OPT_TENSOR_CORES = 1
+};
+
+/* Set an option of the plan (see enum spectre_option).  Takes effect for
+ * runs enqueued afterwards.  SPECTRE_ERR_ARG for a NULL handle, an unknown
+ * option or a value out of range. */
+int spectre_mix_set_option(spectre_mix_t h, int option, int value);
+
+/*
+ * Synchronise `stream` and report device-side failures of the handle's
+ * earlier runs: SPECTRE_ERR_TIMEOUT if a bounded wait for a tensor-core MMA
+ * gave up in any run since the last call (those runs' outputs are invalid),
+ * else SPECTRE_OK.  Clears the recorded failure.
+ */
+int spectre_mix_device_status(spectre_mix_t h, void *stream);
 
 /* Free the handle, its tables, workspace and staging buffers.  NULL-safe.
  * Synchronises the device the handle lives on before freeing. */

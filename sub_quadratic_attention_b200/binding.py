@@ -24,6 +24,9 @@ SPECTRE_ERR_CUDA = -4
 SPECTRE_ERR_NOMEM = -5
 SPECTRE_ERR_DEVICE = -6
 SPECTRE_ERR_SCRATCH = -7
+SPECTRE_ERR_TIMEOUT = -8
+
+SPECTRE_OPT_TENSOR_CORES = 1
 
 # fixed device scratch behind spectre_mix_run_noalloc (SPECTRE_NOALLOC_SCRATCH_BYTES)
 SPECTRE_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -39,6 +42,8 @@ SIGNATURES = {
     "spectre_mix_run_profiled": (_i, [_vp] * 10 + [_i, _vp]),
     "spectre_mix_run_noalloc": (_i, [_i] * 6 + [ctypes.c_float] + [_vp] * 9),
     "spectre_mix_destroy": (_i, [_vp]),
+    "spectre_mix_device_status": (_i, [_vp, _vp]),
+    "spectre_mix_set_option": (_i, [_vp, _i, _i]),
     "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
     "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
     "spectre_mix_plan_info": (_i, [_vp] + [ctypes.POINTER(_i)] * 5),
@@ -157,6 +162,15 @@ def spectre_mix_run_noalloc(B: int, L: int, H: int, D: int, F: int, dtype: int, 
                                           y, stream), "spectre_mix_run_noalloc")
 
 
+def spectre_mix_set_option(h: int, option: int, value: int) -> None:
+    _check(_lib.spectre_mix_set_option(h, option, value), "spectre_mix_set_option")
+
+
+def spectre_mix_device_status(h: int, stream=None) -> int:
+    """Synchronise and return SPECTRE_OK or SPECTRE_ERR_TIMEOUT for earlier runs."""
+    return _lib.spectre_mix_device_status(h, _stream(stream))
+
+
 def spectre_mix_destroy(h: Optional[int]) -> None:
     _check(_lib.spectre_mix_destroy(h), "spectre_mix_destroy")
 
@@ -180,13 +194,15 @@ class SpectreMix:
     """
 
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
-                 dtype: str = "bf16", eps: float = 1e-5):
+                 dtype: str = "bf16", eps: float = 1e-5, tensor_cores: bool = False):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
         self.F = L // 2 + 1 if F is None else F
         self.dtype_code = SPECTRE_F32 if dtype in ("f32", "float32", "fp32") else SPECTRE_BF16
         self.eps = eps
         self.handle = spectre_mix_create(B, L, H, D, self.F, self.dtype_code, eps)
+        if tensor_cores:
+            spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1)
 
     def __call__(self, q, k, v, x, G, gamma, beta, y=None, out=None, stream=None):
         import torch

@@ -24,6 +24,7 @@ struct PathGeom {
     int p16;             // P stored as fp16 with per-slice scales (bf16 I/O)
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
+    int use_tc;          // option: length-16 DFT stages on the tensor cores
     size_t a_bytes, p_bytes, s_bytes;
 };
 
@@ -34,6 +35,7 @@ struct PathBuffers {
     float2 *A;           // [3][B][W][NF][M]
     void *P;             // [B][C][NF][M] float2 or __half2
     float *pscale;       // [B][C][NF]
+    int *err;            // device error word (bit 0: a tensor-core wait timed out)
 };
 
 struct spectre_mix_s {
@@ -166,10 +168,11 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
         while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
     }
     g->T2C = T2C;
+    g->use_tc = 0;
     const size_t slices = (size_t)B * C * NF;
     g->a_bytes = align_up((size_t)3 * B * W * NF * M * sizeof(float2), 256);
     g->p_bytes = align_up(slices * M * (g->p16 ? 4 : 8), 256);
-    g->s_bytes = align_up(slices * sizeof(float), 256);
+    g->s_bytes = align_up(slices * sizeof(float), 256) + 256;   // scales, then the error word
     return SPECTRE_OK;
 }
 
@@ -205,6 +208,8 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
         sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
         sa.c_lo = c_lo; sa.Cw = Cw;
         sa.p16 = g.p16;
+        sa.use_tc = (g.use_tc && g.p16 && g.M == 4096) ? 1 : 0;
+        sa.err = bf.err;
         sa.nbins = g.L / 2 + 1;
         sa.nslices = (long long)g.B * Cw * g.NF;
         sa.invL = 1.0f / (float)g.L;
@@ -249,6 +254,7 @@ const char *spectre_mix_error_string(int code) {
     case SPECTRE_ERR_NOMEM: return "out of memory";
     case SPECTRE_ERR_DEVICE: return "no usable sm_100 device, or the handle's device is not current";
     case SPECTRE_ERR_SCRATCH: return "problem needs more than the 64 MiB no-allocation scratch holds";
+    case SPECTRE_ERR_TIMEOUT: return "a bounded wait on the tensor cores timed out; results of the run are invalid";
     default: return "unknown status";
     }
 }
@@ -334,6 +340,13 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     h->bufs.A = reinterpret_cast<float2 *>(base);
     h->bufs.P = base + g.a_bytes;
     h->bufs.pscale = reinterpret_cast<float *>(base + g.a_bytes + g.p_bytes);
+    h->bufs.err = reinterpret_cast<int *>(base + g.a_bytes + g.p_bytes + g.s_bytes - 256);
+    e = cudaMemset(h->bufs.err, 0, sizeof(int));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        free_handle(h);
+        return cuda_status(e);
+    }
     *out = h;
     return SPECTRE_OK;
 }
@@ -484,6 +497,7 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     bf.A = reinterpret_cast<float2 *>(base + tab_bytes);
     bf.P = base + tab_bytes + g.a_bytes;
     bf.pscale = reinterpret_cast<float *>(base + tab_bytes + g.a_bytes + g.p_bytes);
+    bf.err = nullptr;   // no error word: the no-allocation path reports launch errors only
     {
         int si = 1;
         for (int d = 0; d < 2; d++)
@@ -493,6 +507,37 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     e = launch_make_tables(tw, segs, s);
     if (e != cudaSuccess) return cuda_status(e);
     return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s);
+}
+
+int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
+    if (!h) return SPECTRE_ERR_ARG;
+    switch (option) {
+    case SPECTRE_OPT_TENSOR_CORES:
+        if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
+        h->g.use_tc = value;
+        return SPECTRE_OK;
+    default: return SPECTRE_ERR_ARG;
+    }
+}
+
+int spectre_mix_device_status(spectre_mix_t h, void *stream) {
+    if (!h) return SPECTRE_ERR_ARG;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) {
+        cudaGetLastError();
+        return SPECTRE_ERR_DEVICE;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, h->bufs.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && word != 0) e = cudaMemsetAsync(h->bufs.err, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_status(e);
+    }
+    return word ? SPECTRE_ERR_TIMEOUT : SPECTRE_OK;
 }
 
 int spectre_mix_destroy(spectre_mix_t h) {

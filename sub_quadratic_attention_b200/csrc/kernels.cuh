@@ -50,6 +50,8 @@ struct SliceArgs {
     int B, L, R, M, C, D, F, nbins;
     int c_lo, Cw;         // channel wave
     int p16;              // store P as fp16 with a power-of-two scale per slice
+    int use_tc;           // length-16 DFT stages on the tensor cores (M = 4096)
+    int *err;             // device error word: bit 0 = a tensor-core wait timed out
     long long nslices;    // B * Cw * (R/2+1)
     float invL;
 };

@@ -18,17 +18,19 @@ def to_device(inputs):
     return {k: v.cuda() for k, v in inputs.items()}
 
 
-def run_library(w, inputs_cpu, debug=True, stream=None):
+def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=False):
     """Run the CUDA path through the C ABI.  Returns (out_f32 or None, y) on CPU."""
+    from sub_quadratic_attention_b200 import binding
     from sub_quadratic_attention_b200.binding import SpectreMix
 
     d = to_device(inputs_cpu)
-    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps) as mix:
+    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps, tensor_cores=tensor_cores) as mix:
         y = torch.empty_like(d["x"])
         out = torch.empty((w.B, w.L, w.C), dtype=torch.float32, device="cuda") if debug else None
         mix(d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y=y, out=out,
             stream=stream)
         torch.cuda.synchronize()
+        assert binding.spectre_mix_device_status(mix.handle) == binding.SPECTRE_OK
     return (out.cpu() if debug else None), y.cpu()
 
 

@@ -58,6 +58,18 @@ def test_shape_sweep_bf16(B, L, H, D, F):
     check_parity(w, out, y, out_ref, y_ref)
 
 
+@pytest.mark.parametrize("case", ["bf16_long", (1, 65536, 2, 8, 8192), (2, 65536, 3, 5, 32769)])
+def test_tensor_core_variant(case):
+    """The slice pass with its length-16 DFT stages on the tensor cores
+    (fp16 operands, fp32 accumulation) meets the bf16 bar as well."""
+    w = WORKLOADS[case] if isinstance(case, str) else custom(*case, dtype="bf16")
+    inp = make_inputs(w)
+    out, y = run_library(w, inp, tensor_cores=True)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"tensor cores {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
 def test_zero_gate_gives_layernorm_of_x():
     w = custom(2, 4096, 4, 16, 2049, dtype="f32")
     inp = make_inputs(w)
