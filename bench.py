@@ -232,11 +232,12 @@ def native_arm(args, w, rank, world, local_rank):
     import torch.distributed as dist
 
     from sub_quadratic_attention_b200 import binding
+    from sub_quadratic_attention_b200.ranks import job_throughput, max_over_ranks, rank_seed_offset
     from sub_quadratic_attention_b200.workloads import make_inputs
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    inputs = make_inputs(w, seed_offset=rank)
+    inputs = make_inputs(w, seed_offset=rank_seed_offset(rank))
     d = {k: v.to(dev) for k, v in inputs.items()}
     y = torch.empty_like(d["x"])
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -288,14 +289,10 @@ def native_arm(args, w, rank, world, local_rank):
         for i in range(nlaunch):
             kind = 2 if i == nlaunch - 1 else (i % 2)
             kern_ms[kind][s_i] += e[i].elapsed_time(e[i + 1])
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = w.B * w.L * world
-    value = tokens_per_step / (ms_per_step * 1e-3)
+    value = job_throughput(w.B * w.L, world, args.steps, total_ms)
 
     # ---- end-to-end through the host-buffer entry point
     pinned = {k: v.pin_memory() for k, v in inputs.items()}
@@ -315,12 +312,8 @@ def native_arm(args, w, rank, world, local_rank):
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_total = sum(e[0].elapsed_time(e[1]) for e in e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = tokens_per_step / (e2e_total / args.steps * 1e-3)
+    e2e_total = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev), dev)
+    e2e_value = job_throughput(w.B * w.L, world, args.steps, e2e_total)
     nelem = w.B * w.L * w.C
     h2d = 4 * nelem * w.elem_bytes + inputs["G"].numel() * 4 + 2 * w.C * 4
     d2h = nelem * w.elem_bytes
