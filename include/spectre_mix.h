@@ -27,8 +27,11 @@
  * bf16 is rounded to nearest even.
  *
  * Ownership: the caller owns every tensor.  The handle owns its twiddle
- * tables and its workspace (allocated by spectre_mix_create, freed by
- * spectre_mix_destroy).
+ * tables, its workspace, one auxiliary CUDA stream and two events (created
+ * by spectre_mix_create, released by spectre_mix_destroy).  spectre_mix_run
+ * forks that stream from the caller's stream and joins it back before it
+ * returns control of the work to `stream`, so stream ordering for the caller
+ * is unchanged.
  *
  * Errors: every function returns a status code (SPECTRE_OK or a negative
  * SPECTRE_ERR_*), never throws and never exits.  Device faults of an
@@ -120,9 +123,12 @@ int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k,
 /*
  * As spectre_mix_run, and also records CUDA events on `stream` around every
  * kernel launch of the path, for per-kernel timing.  The path is, for each
- * channel wave w (see spectre_mix_plan_info), a row-pass launch then a
- * slice-pass launch, and finally one inverse-row-pass launch: n launches in
- * all.  `events` points to nevents = n + 1 cudaEvent_t created by the caller;
+ * channel chunk, a row-pass launch then a slice-pass launch, and finally one
+ * inverse-row-pass launch: n launches in all (see spectre_mix_plan_info).
+ * spectre_mix_run overlaps one chunk's row pass with the previous chunk's
+ * slice pass on a second stream the handle owns; the profiled run keeps all
+ * launches on `stream`, one after another, so each event pair brackets one
+ * kernel.  `events` points to nevents = n + 1 cudaEvent_t created by the caller;
  * events[i] is recorded before launch i and events[n] after the last.
  * Returns SPECTRE_ERR_ARG if nevents != n + 1 or an event is NULL.
  */

@@ -25,6 +25,7 @@ struct PathGeom {
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
     int use_tc;          // option: length-16 DFT stages on the tensor cores
+    int chunk;           // channels per pipeline chunk (multiple of 64, or C)
     size_t a_bytes, p_bytes, s_bytes;
 };
 
@@ -41,6 +42,10 @@ struct PathBuffers {
 struct spectre_mix_s {
     int device;
     PathGeom g;
+    // second stream and fork/join events: the row pass of one channel chunk
+    // overlaps the slice pass of the previous chunk
+    cudaStream_t aux;
+    cudaEvent_t ev_fork, ev_join;
     // device memory owned by the handle
     void *tables;       // twL followed by the slice tables
     void *ws;           // A, P, pscale
@@ -113,6 +118,9 @@ int check_device(int *dev_out) {
 
 void free_handle(spectre_mix_s *h) {
     if (!h) return;
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->aux) cudaStreamDestroy(h->aux);
     if (h->tables) cudaFree(h->tables);
     if (h->ws) cudaFree(h->ws);
     if (h->stage) cudaFree(h->stage);
@@ -169,6 +177,9 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     }
     g->T2C = T2C;
     g->use_tc = 0;
+    // pipeline chunks: four channel chunks when each still fills the GPU
+    g->chunk = C;
+    if (W == C && C >= 256) g->chunk = (int)align_up((size_t)(C + 3) / 4, 64);
     const size_t slices = (size_t)B * C * NF;
     g->a_bytes = align_up((size_t)3 * B * W * NF * M * sizeof(float2), 256);
     g->p_bytes = align_up(slices * M * (g->p16 ? 4 : 8), 256);
@@ -176,45 +187,65 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     return SPECTRE_OK;
 }
 
-int wave_count(const PathGeom &g) { return (g.C + g.W - 1) / g.W; }
-
-// The launch sequence of one mix: per channel wave the row pass then the
-// slice pass, then the inverse row pass with residual + LayerNorm.  events
-// (nullable, 2 * waves + 2 of them) are recorded before every launch and
-// after the last.
+// The launch sequence of one mix.  Per channel chunk (within each wave) the
+// row pass then the slice pass, then the inverse row pass with residual +
+// LayerNorm.  Each chunk has its own region of A, so with an auxiliary stream
+// the chunks alternate between `s` and `aux` and the row pass of chunk k + 1
+// runs while the slice pass of chunk k does; `aux` forks from and joins back
+// into `s`.  events (nullable, one per launch + 1) are recorded before every
+// launch and after the last; with events the schedule is single-stream.
 int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const void *k, const void *v,
                 const void *x, const float *G, const float *gamma, const float *beta, void *y,
-                float *out_f32, void *const *events, cudaStream_t s) {
+                float *out_f32, void *const *events, cudaStream_t s, cudaStream_t aux,
+                cudaEvent_t ev_fork, cudaEvent_t ev_join) {
     int ev = 0;
-    auto mark = [&]() -> cudaError_t {
-        return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s) : cudaSuccess;
+    auto mark = [&](cudaStream_t st) -> cudaError_t {
+        return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), st) : cudaSuccess;
     };
+    const bool two = aux && !events && g.chunk < g.W;
     cudaError_t e = cudaSuccess;
-    for (int c_lo = 0; c_lo < g.C; c_lo += g.W) {
-        const int Cw = g.C - c_lo < g.W ? g.C - c_lo : g.W;
-        RowsFwdArgs fa;
-        fa.q = q; fa.k = k; fa.v = v;
-        fa.A = bf.A;
-        fa.twL = bf.twL;
-        fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
-        fa.c_lo = c_lo; fa.Cw = Cw;
-        fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
-        e = mark();
-        if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, s);
+    if (two) {
+        e = cudaEventRecord(ev_fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(aux, ev_fork, 0);
         if (e != cudaSuccess) return cuda_status(e);
+    }
+    int idx = 0;
+    for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
+        const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
+        for (int c_lo = w_lo; c_lo < w_hi; c_lo += g.chunk, idx++) {
+            const int Cw = w_hi - c_lo < g.chunk ? w_hi - c_lo : g.chunk;
+            cudaStream_t st = (two && (idx & 1)) ? aux : s;
+            // this chunk's region of A: [3][B][Cw][NF][M] at its offset in the wave
+            float2 *A = bf.A + (size_t)3 * g.B * (c_lo - w_lo) * g.NF * g.M;
+            RowsFwdArgs fa;
+            fa.q = q; fa.k = k; fa.v = v;
+            fa.A = A;
+            fa.twL = bf.twL;
+            fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
+            fa.c_lo = c_lo; fa.Cw = Cw;
+            fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
+            e = mark(st);
+            if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, st);
+            if (e != cudaSuccess) return cuda_status(e);
 
-        SliceArgs sa;
-        sa.A = bf.A; sa.P = bf.P; sa.pscale = bf.pscale; sa.twL = bf.twL; sa.G = G; sa.tabs = bf.tabs;
-        sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
-        sa.c_lo = c_lo; sa.Cw = Cw;
-        sa.p16 = g.p16;
-        sa.use_tc = (g.use_tc && g.p16 && g.M == 4096) ? 1 : 0;
-        sa.err = bf.err;
-        sa.nbins = g.L / 2 + 1;
-        sa.nslices = (long long)g.B * Cw * g.NF;
-        sa.invL = 1.0f / (float)g.L;
-        e = mark();
-        if (e == cudaSuccess) e = launch_slices(sa, s);
+            SliceArgs sa;
+            sa.A = A; sa.P = bf.P; sa.pscale = bf.pscale; sa.twL = bf.twL; sa.G = G; sa.tabs = bf.tabs;
+            sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
+            sa.c_lo = c_lo; sa.Cw = Cw;
+            sa.p16 = g.p16;
+            sa.use_tc = (g.use_tc && g.p16 && g.M == 4096) ? 1 : 0;
+            sa.err = bf.err;
+            sa.nbins = g.L / 2 + 1;
+            sa.nslices = (long long)g.B * Cw * g.NF;
+            sa.invL = 1.0f / (float)g.L;
+            e = mark(st);
+            if (e == cudaSuccess) e = launch_slices(sa, st);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+    }
+    if (two) {
+        e = cudaEventRecord(ev_join, aux);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_join, 0);
         if (e != cudaSuccess) return cuda_status(e);
     }
     RowsInvArgs ia;
@@ -224,11 +255,20 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     ia.T2C = g.T2C; ia.ZS = g.ZS; ia.eps = g.eps;
     ia.reg_variant = g.inv_reg;
     ia.vec2 = (g.C % 2 == 0) ? 1 : 0;
-    e = mark();
+    e = mark(s);
     if (e == cudaSuccess) e = launch_rows_inv_ln(g.R, g.dtype, ia, s);
-    if (e == cudaSuccess) e = mark();
+    if (e == cudaSuccess) e = mark(s);
     if (e != cudaSuccess) return cuda_status(e);
     return SPECTRE_OK;
+}
+
+int launch_count(const PathGeom &g) {
+    int n = 0;
+    for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
+        const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
+        n += 2 * ((w_hi - w_lo + g.chunk - 1) / g.chunk);
+    }
+    return n + 1;
 }
 
 size_t l2_size(int dev) {
@@ -342,6 +382,11 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     h->bufs.pscale = reinterpret_cast<float *>(base + g.a_bytes + g.p_bytes);
     h->bufs.err = reinterpret_cast<int *>(base + g.a_bytes + g.p_bytes + g.s_bytes - 256);
     e = cudaMemset(h->bufs.err, 0, sizeof(int));
+    if (e == cudaSuccess && g.chunk < g.W) {
+        e = cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    }
     if (e != cudaSuccess) {
         cudaGetLastError();
         free_handle(h);
@@ -366,7 +411,7 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
     }
     if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
     return launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, out_f32, events,
-                       static_cast<cudaStream_t>(stream));
+                       static_cast<cudaStream_t>(stream), h->aux, h->ev_fork, h->ev_join);
 }
 
 int spectre_mix_run(spectre_mix_t h, const void *q, const void *k, const void *v, const void *x,
@@ -384,7 +429,7 @@ int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k, cons
                              const void *x, const float *G, const float *gamma, const float *beta,
                              void *y, void *const *events, int nevents, void *stream) {
     if (!h || !events) return SPECTRE_ERR_ARG;
-    const int need = 2 * wave_count(h->g) + 2;
+    const int need = launch_count(h->g) + 1;
     if (nevents != need) return SPECTRE_ERR_ARG;
     for (int i = 0; i < need; i++)
         if (!events[i]) return SPECTRE_ERR_ARG;
@@ -506,7 +551,9 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     }
     e = launch_make_tables(tw, segs, s);
     if (e != cudaSuccess) return cuda_status(e);
-    return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s);
+    // single stream: this path creates no streams or events
+    return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s, nullptr, nullptr,
+                       nullptr);
 }
 
 int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
@@ -567,7 +614,7 @@ int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_chann
     if (M) *M = h->g.M;
     if (slices_per_channel) *slices_per_channel = h->g.NF;
     if (channels_per_wave) *channels_per_wave = h->g.W;
-    if (launches) *launches = 2 * wave_count(h->g) + 1;
+    if (launches) *launches = launch_count(h->g);
     return SPECTRE_OK;
 }
 

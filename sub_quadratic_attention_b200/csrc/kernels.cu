@@ -64,7 +64,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // A, straight from registers.
 // ---------------------------------------------------------------------------
 template <int R, typename T>
-__global__ void __launch_bounds__(256, R <= 16 ? 3 : 1) spectre_rows_fwd(RowsFwdArgs a) {
+__global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwdArgs a) {
     constexpr int NF = R / 2 + 1;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t2 = blockIdx.x * 8 + (warp & 1) * 4 + (lane & 3);
