@@ -243,7 +243,7 @@ def native_arm(args, w, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps,
-                             tensor_cores=args.tensor_cores)
+                             tensor_cores=False if args.cuda_core_slices else None)
     h = mix.handle
 
     def barrier():
@@ -356,7 +356,7 @@ def native_arm(args, w, rank, world, local_rank):
                         "row pass with the previous chunk's slice pass on two streams",
         "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
                  "chunks": nchunks, "launches_per_step": nlaunch,
-                 "tensor_core_dft16": bool(args.tensor_cores)},
+                 "slice_pass": mix.slice_pass},
     }
 
     # ---- CPU baseline (rank 0, N = 1 only)
@@ -404,8 +404,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tensor-cores", action="store_true",
-                    help="run the slice pass's DFT16 stages on tcgen05 (plan option)")
+    ap.add_argument("--cuda-core-slices", action="store_true",
+                    help="force the CUDA-core slice pass (plan option; default: tensor cores "
+                         "where the plan allows)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -172,12 +172,14 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype,
                             void *stream);
 
 enum spectre_option {
-    /* 0 (default): the slice pass's length-16 DFT stages run as CUDA-core
-     * butterflies.  1: they run on the tensor cores (tcgen05 MMA with fp16
-     * operands and fp32 accumulation against a DFT16/16 matrix), for bf16 I/O
-     * plans whose slice length M is 4096; other plans ignore the option.
-     * Measured on B200 for the bf16 long workload the tensor-core variant is
-     * slower (each stage waits for its MMA), hence the default. */
+    /* 1 (default): plans with bf16 I/O, slice length M = 4096 (L = 65536) and
+     * a truncation that leaves at most 16 live bins per slice row (F <= L/8
+     * roughly) run the slice pass on the tensor cores: every 4096-point
+     * transform as two DFT-64 passes of tcgen05 MMAs with fp16 operands
+     * (power-of-two scaled per slice) and fp32 accumulation in tensor memory,
+     * the truncation pruning the MMAs.  0: the CUDA-core slice pass (fp32
+     * Stockham radix-16 butterflies) for every plan.  Plans outside the
+     * tensor-core range always take the CUDA-core pass. */
     SPECTRE_OPT_TENSOR_CORES = 1
 };
 
@@ -185,6 +187,15 @@ enum spectre_option {
  * runs enqueued afterwards.  SPECTRE_ERR_ARG for a NULL handle, an unknown
  * option or a value out of range. */
 int spectre_mix_set_option(spectre_mix_t h, int option, int value);
+
+enum spectre_slice_pass {
+    SPECTRE_SLICE_CUDA_CORES = 0,
+    SPECTRE_SLICE_TENSOR_CORES = 1
+};
+
+/* Which slice pass runs of the plan launch under its current options
+ * (enum spectre_slice_pass); SPECTRE_ERR_ARG for a NULL handle. */
+int spectre_mix_slice_pass(spectre_mix_t h);
 
 /*
  * Synchronise `stream` and report device-side failures of the handle's

@@ -28,6 +28,9 @@ SPECTRE_ERR_TIMEOUT = -8
 
 SPECTRE_OPT_TENSOR_CORES = 1
 
+SPECTRE_SLICE_CUDA_CORES = 0
+SPECTRE_SLICE_TENSOR_CORES = 1
+
 # fixed device scratch behind spectre_mix_run_noalloc (SPECTRE_NOALLOC_SCRATCH_BYTES)
 SPECTRE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -44,6 +47,7 @@ SIGNATURES = {
     "spectre_mix_destroy": (_i, [_vp]),
     "spectre_mix_device_status": (_i, [_vp, _vp]),
     "spectre_mix_set_option": (_i, [_vp, _i, _i]),
+    "spectre_mix_slice_pass": (_i, [_vp]),
     "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
     "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
     "spectre_mix_plan_info": (_i, [_vp] + [ctypes.POINTER(_i)] * 5),
@@ -166,6 +170,14 @@ def spectre_mix_set_option(h: int, option: int, value: int) -> None:
     _check(_lib.spectre_mix_set_option(h, option, value), "spectre_mix_set_option")
 
 
+def spectre_mix_slice_pass(h: int) -> int:
+    """SPECTRE_SLICE_TENSOR_CORES or SPECTRE_SLICE_CUDA_CORES for the plan's runs."""
+    st = _lib.spectre_mix_slice_pass(h)
+    if st < 0:
+        _check(st, "spectre_mix_slice_pass")
+    return st
+
+
 def spectre_mix_device_status(h: int, stream=None) -> int:
     """Synchronise and return SPECTRE_OK or SPECTRE_ERR_TIMEOUT for earlier runs."""
     return _lib.spectre_mix_device_status(h, _stream(stream))
@@ -194,15 +206,15 @@ class SpectreMix:
     """
 
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
-                 dtype: str = "bf16", eps: float = 1e-5, tensor_cores: bool = False):
+                 dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
         self.F = L // 2 + 1 if F is None else F
         self.dtype_code = SPECTRE_F32 if dtype in ("f32", "float32", "fp32") else SPECTRE_BF16
         self.eps = eps
         self.handle = spectre_mix_create(B, L, H, D, self.F, self.dtype_code, eps)
-        if tensor_cores:
-            spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1)
+        if tensor_cores is not None:   # None keeps the library's default (on)
+            spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1 if tensor_cores else 0)
 
     def __call__(self, q, k, v, x, G, gamma, beta, y=None, out=None, stream=None):
         import torch
@@ -226,6 +238,12 @@ class SpectreMix:
     @property
     def plan(self) -> Tuple[int, int, int, int, int]:
         return spectre_mix_plan_info(self.handle)
+
+    @property
+    def slice_pass(self) -> str:
+        """'tensor_cores' or 'cuda_cores': the slice pass runs of this plan launch."""
+        sp = spectre_mix_slice_pass(self.handle)
+        return "tensor_cores" if sp == SPECTRE_SLICE_TENSOR_CORES else "cuda_cores"
 
     def close(self) -> None:
         if self.handle is not None:

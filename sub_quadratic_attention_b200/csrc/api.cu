@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libspectre_mix (declared in include/spectre_mix.h):
 // argument validation, the plan (decomposition, twiddle tables, workspace)
 // and the launch sequence.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -24,7 +25,9 @@ struct PathGeom {
     int p16;             // P stored as fp16 with per-slice scales (bf16 I/O)
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
-    int use_tc;          // option: length-16 DFT stages on the tensor cores
+    int tc_mode;         // option: slice pass on the tensor cores where mma_ok (1) or CUDA cores (0)
+    int mma_ok;          // the DFT-64 MMA slice pass applies (M = 4096, fp16 P, few live groups)
+    int nsm;             // multiprocessors of the device
     int chunk;           // channels per pipeline chunk (multiple of 64, or C)
     size_t a_bytes, p_bytes, s_bytes;
 };
@@ -33,6 +36,8 @@ struct PathGeom {
 struct PathBuffers {
     const float2 *twL;
     SliceTables tabs;
+    const float2 *twMM;  // M = 4096: w_4096^{n2 k1} as [k1][n2]
+    const void *w64op;   // M = 4096: the fp16 DFT-64 operand
     float2 *A;           // [3][B][W][NF][M]
     void *P;             // [B][C][NF][M] float2 or __half2
     float *pscale;       // [B][C][NF]
@@ -176,7 +181,20 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
         while (T2C > 1 && (size_t)R * T2C * ZS * sizeof(float) > 160 * 1024) T2C /= 2;
     }
     g->T2C = T2C;
-    g->use_tc = 0;
+    // tensor-core slice pass: M = 4096 as two DFT-64 MMA passes, for fp16 P,
+    // when no slice has more than kMmaMaxGroups live k2 groups
+    g->mma_ok = 0;
+    if (M == 4096 && g->p16) {
+        int worst = 0;
+        for (int f1 = 0; f1 < NF; f1++) {
+            int n = 0;
+            for (int grp = 0; grp < 8; grp++) n += mma_group_live(grp, f1, R, L, F) ? 1 : 0;
+            worst = n > worst ? n : worst;
+        }
+        g->mma_ok = worst <= kMmaMaxGroups ? 1 : 0;
+    }
+    g->tc_mode = 1;
+    g->nsm = 148;
     // pipeline chunks: four channel chunks when each still fills the GPU
     g->chunk = C;
     if (W == C && C >= 256) g->chunk = (int)align_up((size_t)(C + 3) / 4, 64);
@@ -185,6 +203,20 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     g->p_bytes = align_up(slices * M * (g->p16 ? 4 : 8), 256);
     g->s_bytes = align_up(slices * sizeof(float), 256) + 256;   // scales, then the error word
     return SPECTRE_OK;
+}
+
+// Whether the slice pass runs on the tensor cores (option on and the plan in
+// the tensor-core kernel's range).
+bool uses_mma(const PathGeom &g) { return g.tc_mode == 1 && g.mma_ok; }
+
+// Channels per pipeline chunk.  Measured on B200 for the bf16 long workload:
+// four chunks suit the CUDA-core slice pass (0.573 ms per mix against 0.60 ms
+// unchunked); the tensor-core slice pass, whose blocks each carry a long
+// chain of dependent phases, does best with two (0.454 ms against 0.460 with
+// four and 0.464 unchunked), which keep more blocks per launch.
+int chunk_channels(const PathGeom &g) {
+    if (!uses_mma(g) || g.chunk >= g.W) return g.chunk;
+    return (int)align_up((size_t)(g.C + 1) / 2, 64);
 }
 
 // The launch sequence of one mix.  Per channel chunk (within each wave) the
@@ -202,7 +234,8 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     auto mark = [&](cudaStream_t st) -> cudaError_t {
         return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), st) : cudaSuccess;
     };
-    const bool two = aux && !events && g.chunk < g.W;
+    const int chunk = chunk_channels(g);
+    const bool two = aux && !events && chunk < g.W;
     cudaError_t e = cudaSuccess;
     if (two) {
         e = cudaEventRecord(ev_fork, s);
@@ -212,8 +245,8 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     int idx = 0;
     for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
         const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
-        for (int c_lo = w_lo; c_lo < w_hi; c_lo += g.chunk, idx++) {
-            const int Cw = w_hi - c_lo < g.chunk ? w_hi - c_lo : g.chunk;
+        for (int c_lo = w_lo; c_lo < w_hi; c_lo += chunk, idx++) {
+            const int Cw = w_hi - c_lo < chunk ? w_hi - c_lo : chunk;
             cudaStream_t st = (two && (idx & 1)) ? aux : s;
             // this chunk's region of A: [3][B][Cw][NF][M] at its offset in the wave
             float2 *A = bf.A + (size_t)3 * g.B * (c_lo - w_lo) * g.NF * g.M;
@@ -233,7 +266,10 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
             sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
             sa.c_lo = c_lo; sa.Cw = Cw;
             sa.p16 = g.p16;
-            sa.use_tc = (g.use_tc && g.p16 && g.M == 4096) ? 1 : 0;
+            sa.use_mma = uses_mma(g) ? 1 : 0;
+            sa.nsm = g.nsm;
+            sa.twMM = bf.twMM;
+            sa.w64op = bf.w64op;
             sa.err = bf.err;
             sa.nbins = g.L / 2 + 1;
             sa.nslices = (long long)g.B * Cw * g.NF;
@@ -266,7 +302,7 @@ int launch_count(const PathGeom &g) {
     int n = 0;
     for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
         const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
-        n += 2 * ((w_hi - w_lo + g.chunk - 1) / g.chunk);
+        n += 2 * ((w_hi - w_lo + chunk_channels(g) - 1) / chunk_channels(g));
     }
     return n + 1;
 }
@@ -347,6 +383,32 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
             ns *= r;
         }
     }
+    // M = 4096: the twiddles between the two DFT-64 passes and the fp16
+    // DFT-64 operand of the tensor-core slice pass
+    size_t off_mm = 0, off_op = 0;
+    if (M == 4096) {
+        off_mm = align_up(host.size(), 2);
+        host.resize(off_mm);
+        for (int k1 = 0; k1 < 64; k1++)
+            for (int n2 = 0; n2 < 64; n2++) {
+                double ang = -2.0 * M_PI * (double)(n2 * k1) / 4096.0;
+                host.push_back(make_float2((float)std::cos(ang), (float)std::sin(ang)));
+            }
+        off_op = align_up(host.size(), 2);
+        host.resize(off_op + 4096);
+        unsigned char *bytes = reinterpret_cast<unsigned char *>(host.data() + off_op);
+        for (int n = 0; n < 128; n++)
+            for (int kk = 0; kk < 128; kk++) {
+                long long ee;
+                int part;
+                dft64_operand_angle(n, kk, &ee, &part);
+                const double ang = -2.0 * M_PI * (double)ee / 64.0;
+                const double val = (part == 0 || part == 3) ? std::cos(ang)
+                                 : (part == 1 ? -std::sin(ang) : std::sin(ang));
+                const __half hv = __float2half_rn((float)(val / 64.0));
+                std::memcpy(bytes + dft64_operand_offset(n, kk), &hv, sizeof(hv));
+            }
+    }
     float2 w64[64];
     for (int e = 0; e < 64; e++) {
         double ang = -2.0 * M_PI * e / 64.0;
@@ -364,6 +426,14 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
         return cuda_status(e);
     }
     h->bufs.twL = static_cast<float2 *>(h->tables);
+    h->bufs.twMM = M == 4096 ? h->bufs.twL + off_mm : nullptr;
+    h->bufs.w64op = M == 4096 ? static_cast<const void *>(h->bufs.twL + off_op) : nullptr;
+    {
+        int nsm = 0;
+        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
+            h->g.nsm = nsm;
+        cudaGetLastError();
+    }
     for (int d = 0; d < 2; d++)
         for (int p = 0; p < kMaxPasses; p++)
             h->bufs.tabs.tw[d][p] = (p > 0 && p < sch.n) ? h->bufs.twL + offs[d][p] : nullptr;
@@ -524,6 +594,16 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
             ns *= r;
         }
     }
+    long long seg_mm = -1, seg_op = -1;
+    if (g.M == 4096) {
+        size_t base = align_up(n_tab, 2);
+        seg_mm = segs.n;
+        segs.seg[segs.n++] = TableSeg{(long long)base, 4096, 64, 4096};
+        base = align_up(base + 4096, 2);
+        seg_op = segs.n;
+        segs.seg[segs.n++] = TableSeg{(long long)base, 4096, -1, 64};
+        n_tab = base + 4096;
+    }
     const size_t tab_bytes = align_up(n_tab * sizeof(float2), 256);
     const size_t need = tab_bytes + g.a_bytes + g.p_bytes + g.s_bytes;
     if (need > kNoAllocScratchBytes) return SPECTRE_ERR_SCRATCH;
@@ -543,6 +623,14 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     bf.P = base + tab_bytes + g.a_bytes;
     bf.pscale = reinterpret_cast<float *>(base + tab_bytes + g.a_bytes + g.p_bytes);
     bf.err = nullptr;   // no error word: the no-allocation path reports launch errors only
+    bf.twMM = seg_mm >= 0 ? tw + segs.seg[seg_mm].offset : nullptr;
+    bf.w64op = seg_op >= 0 ? static_cast<const void *>(tw + segs.seg[seg_op].offset) : nullptr;
+    {
+        int nsm = 0;
+        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
+            g.nsm = nsm;
+        cudaGetLastError();
+    }
     {
         int si = 1;
         for (int d = 0; d < 2; d++)
@@ -561,10 +649,15 @@ int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     switch (option) {
     case SPECTRE_OPT_TENSOR_CORES:
         if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
-        h->g.use_tc = value;
+        h->g.tc_mode = value;
         return SPECTRE_OK;
     default: return SPECTRE_ERR_ARG;
     }
+}
+
+int spectre_mix_slice_pass(spectre_mix_t h) {
+    if (!h) return SPECTRE_ERR_ARG;
+    return uses_mma(h->g) ? SPECTRE_SLICE_TENSOR_CORES : SPECTRE_SLICE_CUDA_CORES;
 }
 
 int spectre_mix_device_status(spectre_mix_t h, void *stream) {

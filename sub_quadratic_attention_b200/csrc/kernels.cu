@@ -17,7 +17,6 @@
 
 #include "fft_regs.cuh"
 #include "kernels.cuh"
-#include "tc_dft.cuh"
 
 namespace spectre {
 
@@ -420,257 +419,6 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
 }
 
 // ---------------------------------------------------------------------------
-// slice pass on the tensor cores (M = 4096 = 16^3, bf16 I/O).  The Stockham
-// structure, the gated product and the stores are those of spectre_slices;
-// each radix-16 butterfly's length-16 DFT runs as one row of a tcgen05 MMA
-// (tc_dft.cuh): thread j = butterfly j writes its 16 twiddled inputs in fp16
-// to row j of an operand tile, one thread issues the MMAs (two 128-row tiles,
-// K = 32 in two steps) and commits them to an mbarrier, and every thread
-// reads its row of the fp32 result back from tensor memory.
-// Scaling: the tile holds values of magnitude <= 2^12 (a per-slice power of
-// two s chosen from the slice's largest input), the DFT matrix carries 1/16,
-// so after the three stages the transform is recovered as result * 4096 / s.
-// Every mbarrier wait is bounded; a timeout sets a device error word and the
-// block stops after releasing its tensor memory.
-// ---------------------------------------------------------------------------
-constexpr uint32_t kTcWaitLimit = 1u << 12;   // polls of up to 1 ms each
-
-struct TcSlice {
-    unsigned char *a_tile;   // aliases buf: 256 rows x 64 bytes
-    unsigned char *b_tile;
-    int *flag;               // shared: set when the polling lane gave up
-    uint32_t mbar, taddr, phase;
-    int j;
-    bool bad;
-    // length-16 DFT / 16 of v (times s on the way in when SCALED), in place.
-    // One lane polls the MMA's mbarrier; the others wait at the block barrier.
-    template <bool SCALED>
-    __device__ __forceinline__ void dft(float2 (&v)[16], float s) {
-        tc::put_row<SCALED>(a_tile, j, v, s);
-        tc::fence_proxy_async();
-        tc::fence_before();
-        __syncthreads();
-        if (j == 0) {
-            tc::fence_after();
-            const uint32_t a0 = tc::smem_u32(a_tile), b0 = tc::smem_u32(b_tile);
-            // rows 0..127 -> columns taddr + [0, 32), rows 128..255 -> + [32, 64)
-#pragma unroll
-            for (int t = 0; t < 2; t++)
-#pragma unroll
-                for (int ks = 0; ks < 2; ks++)
-                    tc::mma_f16(taddr + 32 * t, tc::make_desc(a0 + t * tc::kRowTile + ks * 256),
-                                tc::make_desc(b0 + ks * 256), ks);
-            tc::commit(mbar);
-            if (!tc::mbar_wait(mbar, phase, kTcWaitLimit)) *flag = 1;
-        }
-        phase ^= 1u;
-        const bool ok = __syncthreads_and(*flag == 0);
-        tc::fence_after();
-        if (ok) {
-            float d[32];
-            const int w = threadIdx.x >> 5;
-            tc::tmem_ld32(taddr + ((uint32_t)(32 * (w & 3)) << 16) + 32 * (w >> 2), d);
-#pragma unroll
-            for (int r = 0; r < 16; r++) v[r] = make_float2(d[2 * r], d[2 * r + 1]);
-        } else {
-            bad = true;
-        }
-        tc::fence_before();
-    }
-};
-
-// block-wide max of non-negative values through a shared slot (zeroed at start)
-__device__ __forceinline__ float block_max(int *slot, float local) {
-    atomicMax(slot, __float_as_int(local));
-    __syncthreads();
-    return __int_as_float(*slot);
-}
-
-// power of two s with max * s in [2^11, 2^12); 1 for max == 0
-__device__ __forceinline__ float tc_in_scale(float m) {
-    int e = 0;
-    if (m > 0.f) frexpf(m, &e);
-    return ldexpf(1.0f, max(-126, min(126, 12 - e)));
-}
-
-__global__ void __launch_bounds__(256, 3) spectre_slices_tc4096(SliceArgs a) {
-    constexpr int M = 4096, NT = 256;
-    extern __shared__ float4 smem_f4[];
-    float2 *buf = reinterpret_cast<float2 *>(smem_f4);              // 4352 float2 (padded)
-    float2 *sbuf = buf + (M + M / 16);                               // 4096 float2
-    unsigned char *b_tile = reinterpret_cast<unsigned char *>(sbuf + M);   // 2 KB
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(b_tile + 2048);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
-    int *slots = reinterpret_cast<int *>(tslot + 1);                // 6 max slots, 1 flag
-    const int j = threadIdx.x;
-    const int warp = j >> 5;
-    if (warp == 0) tc::tmem_alloc(tslot, 64);
-    if (j == 0) tc::mbar_init(tc::smem_u32(mbar), 1);
-    if (j < 7) slots[j] = 0;
-    tc::fill_dft16_operand(b_tile);
-    tc::fence_before();
-    __syncthreads();
-    tc::fence_after();
-
-    TcSlice tcs;
-    tcs.a_tile = reinterpret_cast<unsigned char *>(buf);
-    tcs.b_tile = b_tile;
-    tcs.flag = &slots[6];
-    tcs.mbar = tc::smem_u32(mbar);
-    tcs.taddr = *tslot;
-    tcs.phase = 0;
-    tcs.j = j;
-    tcs.bad = false;
-
-    const long long sid = blockIdx.x;
-    const bool live = sid < a.nslices;
-    const int NF = a.R / 2 + 1;
-    const long long sidc = live ? sid : 0;
-    const int f1 = (int)(sidc % NF);
-    const long long bcl = sidc / NF;
-    const int b = (int)(bcl / a.Cw);
-    const int c = a.c_lo + (int)(bcl % a.Cw);
-    const int h = c / a.D;
-    const size_t sig_stride = (size_t)a.B * a.Cw * NF * M;
-    const float2 *srcA = a.A + (size_t)bcl * NF * M + (size_t)f1 * M;
-    const size_t pslice = ((size_t)b * a.C + c) * NF + f1;
-    PStore ps;
-    ps.dst = a.p16 ? static_cast<void *>(static_cast<__half2 *>(a.P) + pslice * M)
-                   : static_cast<void *>(static_cast<float2 *>(a.P) + pslice * M);
-    ps.pscale = a.pscale + pslice;
-    ps.smax = &slots[5];
-    ps.live = live;
-    ps.p16 = a.p16 != 0;
-    const float *Gh = a.G + (size_t)h * a.nbins;
-    const float2 *tw1 = a.tabs.tw[0][1], *tw2 = a.tabs.tw[0][2];
-    const float2 *iw1 = a.tabs.tw[1][1], *iw2 = a.tabs.tw[1][2];
-
-    float2 v[16];
-    bool abort = false;   // block-uniform: some tensor-core wait timed out
-    do {
-        // three forward transforms; thread j ends with X[j + 256 r]
-#pragma unroll 1
-        for (int sig = 0; sig < 3; sig++) {
-            const float2 *src = srcA + sig * sig_stride;
-            float mx = 0.f;
-#pragma unroll
-            for (int r = 0; r < 16; r++) {
-                v[r] = live ? __ldg(src + j + r * NT) : make_float2(0.f, 0.f);
-                mx = fmaxf(mx, fmaxf(fabsf(v[r].x), fabsf(v[r].y)));
-            }
-            const float sin_ = tc_in_scale(block_max(&slots[sig], mx));
-            tcs.dft<true>(v, sin_);
-#pragma unroll
-            for (int r = 0; r < 16; r++) buf[spad(j * 16 + r)] = v[r];
-            if ((abort = __syncthreads_or(tcs.bad))) break;
-            // pass 1 (Ns = 16)
-#pragma unroll
-            for (int r = 0; r < 16; r++) v[r] = buf[spad(j + r * NT)];
-            __syncthreads();
-            {
-                const int kk = j & 15;
-#pragma unroll
-                for (int r = 1; r < 16; r++) v[r] = cmul(v[r], __ldg(tw1 + kk + r * 16));
-            }
-            tcs.dft<false>(v, 1.0f);
-            {
-                const int idxD = (j >> 4) * 256 + (j & 15);
-#pragma unroll
-                for (int r = 0; r < 16; r++) buf[spad(idxD + r * 16)] = v[r];
-            }
-            if ((abort = __syncthreads_or(tcs.bad))) break;
-            // pass 2 (Ns = 256), result stays in registers
-#pragma unroll
-            for (int r = 0; r < 16; r++) v[r] = buf[spad(j + r * NT)];
-            __syncthreads();
-#pragma unroll
-            for (int r = 1; r < 16; r++) v[r] = cmul(v[r], __ldg(tw2 + j + r * NT));
-            tcs.dft<false>(v, 1.0f);
-            const float back = 4096.0f / sin_;
-#pragma unroll
-            for (int r = 0; r < 16; r++) v[r] = cscale(v[r], back);
-            // gated product on bins f = f1 + R (j + 256 r)
-            if (sig == 0) {
-#pragma unroll
-                for (int r = 0; r < 16; r++) {
-                    int f = f1 + a.R * (j + r * NT);
-                    int ff = min(f, a.L - f);
-                    float g = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
-                    sbuf[j + r * NT] = cscale(v[r], g);
-                }
-            } else if (sig == 1) {
-#pragma unroll
-                for (int r = 0; r < 16; r++) sbuf[j + r * NT] = cmulc(sbuf[j + r * NT], v[r]);
-            } else {
-#pragma unroll
-                for (int r = 0; r < 16; r++) v[r] = cmul(sbuf[j + r * NT], v[r]);
-            }
-            if ((abort = __syncthreads_or(tcs.bad))) break;
-        }
-        if (abort) break;
-        // inverse: conj, three forward stages in reversed radix order, conj
-        float mx = 0.f;
-#pragma unroll
-        for (int r = 0; r < 16; r++) {
-            v[r] = cconj(v[r]);
-            mx = fmaxf(mx, fmaxf(fabsf(v[r].x), fabsf(v[r].y)));
-        }
-        const float so = tc_in_scale(block_max(&slots[3], mx));
-        tcs.dft<true>(v, so);
-#pragma unroll
-        for (int r = 0; r < 16; r++) buf[spad(j * 16 + r)] = v[r];
-        if ((abort = __syncthreads_or(tcs.bad))) break;
-#pragma unroll
-        for (int r = 0; r < 16; r++) v[r] = buf[spad(j + r * NT)];
-        __syncthreads();
-        {
-            const int kk = j & 15;
-#pragma unroll
-            for (int r = 1; r < 16; r++) v[r] = cmul(v[r], __ldg(iw1 + kk + r * 16));
-        }
-        tcs.dft<false>(v, 1.0f);
-        {
-            const int idxD = (j >> 4) * 256 + (j & 15);
-#pragma unroll
-            for (int r = 0; r < 16; r++) buf[spad(idxD + r * 16)] = v[r];
-        }
-        if ((abort = __syncthreads_or(tcs.bad))) break;
-#pragma unroll
-        for (int r = 0; r < 16; r++) v[r] = buf[spad(j + r * NT)];
-        __syncthreads();
-#pragma unroll
-        for (int r = 1; r < 16; r++) v[r] = cmul(v[r], __ldg(iw2 + j + r * NT));
-        tcs.dft<false>(v, 1.0f);
-        if ((abort = __syncthreads_or(tcs.bad))) break;
-        // P[t2] = w_L^{-f1 t2} * conj(result) at t2 = j + 256 r
-        const float back = 4096.0f / so;
-        float pm = 0.f;
-#pragma unroll
-        for (int r = 0; r < 16; r++) {
-            const int t2 = j + r * NT;
-            v[r] = cconj(cmul(cscale(v[r], back), __ldg(a.twL + f1 * t2)));
-            pm = fmaxf(pm, fmaxf(fabsf(v[r].x), fabsf(v[r].y)));
-        }
-        const float sp = slice_scale(ps, pm);
-#pragma unroll
-        for (int r = 0; r < 16; r++) pstore(ps, j + r * NT, v[r], sp);
-        if (ps.p16 && live && j == 0) {
-            int e = 0;
-            const float m = __int_as_float(slots[5]);
-            if (m > 0.f) frexpf(m, &e);
-            *ps.pscale = ldexpf(1.0f, -max(-126, min(126, 14 - e)));
-        }
-    } while (0);
-    if (abort && j == 0 && a.err) atomicOr(a.err, 1);
-    tc::fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc::fence_after();
-        tc::tmem_dealloc(tcs.taddr, 64);
-    }
-}
-
-// ---------------------------------------------------------------------------
 // inverse row pass + residual + LayerNorm
 // ---------------------------------------------------------------------------
 template <int R, typename T, bool DEBUG_OUT>
@@ -972,13 +720,7 @@ template <int M> static void slice_geom_M(int *nt, int *spb, size_t *smem) {
     X(6144) X(12288)
 
 cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s) {
-    if (a.M == 4096 && a.use_tc) {
-        const size_t smem = (size_t)(4096 + 256 + 4096) * sizeof(float2) + 2048 + 64;
-        cudaFuncSetAttribute(spectre_slices_tc4096, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        spectre_slices_tc4096<<<(unsigned)a.nslices, 256, smem, s>>>(a);
-        return cudaGetLastError();
-    }
+    if (a.M == 4096 && a.use_mma) return launch_slices_mma4096(a, s);
     switch (a.M) {
 #define X(m) case m: return slices_M<m>(a, s);
         SPECTRE_SLICE_LENGTHS(X)
@@ -1105,6 +847,27 @@ __global__ void spectre_make_tables(float2 *base, TableSegs segs) {
     for (int sgi = 0; sgi < segs.n; sgi++) {
         const TableSeg &g = segs.seg[sgi];
         if (i < g.count) {
+            if (g.ns == -1) {
+                // slot i: bytes 8 i .. 8 i + 7 of the DFT-64 operand, four
+                // K-consecutive fp16 values of one row
+                const int byte = 8 * (int)i;
+                const int n = (byte / 2048) * 8 + (byte % 128) / 16;
+                const int k0 = ((byte % 2048) / 128) * 8 + (byte % 16) / 2;
+                __half hv[4];
+                for (int u = 0; u < 4; u++) {
+                    long long e;
+                    int part;
+                    dft64_operand_angle(n, k0 + u, &e, &part);
+                    double sn, cs;
+                    sincospi(-2.0 * (double)e / 64.0, &sn, &cs);
+                    const double val = (part == 0 || part == 3) ? cs : (part == 1 ? -sn : sn);
+                    hv[u] = __float2half_rn((float)(val / 64.0));
+                }
+                float2 slot;
+                memcpy(&slot, hv, sizeof(slot));
+                base[g.offset + i] = slot;
+                return;
+            }
             long long e;
             if (g.ns == 0) {
                 e = i;                                   // w_N^i

@@ -50,8 +50,12 @@ struct SliceArgs {
     int B, L, R, M, C, D, F, nbins;
     int c_lo, Cw;         // channel wave
     int p16;              // store P as fp16 with a power-of-two scale per slice
-    int use_tc;           // length-16 DFT stages on the tensor cores (M = 4096)
-    int *err;             // device error word: bit 0 = a tensor-core wait timed out
+    int use_mma;          // M = 4096 as two DFT-64 passes on the tensor cores
+    int nsm;              // multiprocessors of the device (grid of the MMA slice pass)
+    const float2 *twMM;   // [64][64]: entry k1 * 64 + n2 = w_4096^{n2 k1}
+    const void *w64op;    // DFT-64 / 64 as a 128 x 128 fp16 operand (canonical layout)
+    int *err;             // device error word: bit 0 = a tensor-core wait timed out,
+                          // bit 1 = a slice exceeded the tensor-memory product budget
     long long nslices;    // B * Cw * (R/2+1)
     float invL;
 };
@@ -73,6 +77,7 @@ struct RowsInvArgs {
 // Returns cudaSuccess or the launch error.  dtype: 0 fp32, 1 bf16.
 cudaError_t launch_rows_fwd(int R, int dtype, const RowsFwdArgs &a, cudaStream_t s);
 cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s);
+cudaError_t launch_slices_mma4096(const SliceArgs &a, cudaStream_t s);
 cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStream_t s);
 
 // Slice-transform schedule for length M (radices ascending, largest last).
@@ -116,6 +121,31 @@ constexpr int sched_stride(int M, int d, int p) {
     return ns;
 }
 
+// The tensor-core slice pass (M = 4096) keeps the product of at most this
+// many k2 groups (8 bins of a slice row each) in tensor memory.
+constexpr int kMmaMaxGroups = 2;
+
+// Whether k2 group g (f2 = k1 + 64 k2, k2 in [8 g, 8 g + 8), k1 < 64) of
+// slice f1 holds a bin f = f1 + R f2 with min(f, L - f) < F.
+__host__ __device__ inline bool mma_group_live(int g, int f1, int R, int L, int F) {
+    const long long flo = f1 + (long long)R * (64 * 8 * g);
+    const long long fhi = f1 + (long long)R * (63 + 64 * (8 * g + 7));
+    return flo < F || fhi > (long long)L - F;
+}
+
+// Element (n, k) of the real 128 x 128 form of the DFT-64 matrix / 64:
+// n = 2 o + (0 re | 1 im) indexes outputs, k = 2 i + (0 re | 1 im) inputs,
+// so that out = sum_k B[n][k] in[k] gives (re, im) of sum_i w64^{o i} in_i / 64.
+__host__ __device__ inline void dft64_operand_angle(int n, int k, long long *e, int *part) {
+    *e = (long long)((n >> 1) * (k >> 1)) & 63;      // w64^e
+    *part = ((n & 1) << 1) | (k & 1);                 // 0: Fr, 1: -Fi, 2: Fi, 3: Fr
+}
+// byte offset of (n, k) in the canonical K-major no-swizzle layout with
+// LBO 128 and SBO 2048 (K = 128 fp16 values per row)
+__host__ __device__ inline int dft64_operand_offset(int n, int k) {
+    return (n >> 3) * 2048 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
 // whether M is a supported slice length (2^k <= 16384 or 3*2^k <= 12288)
 bool slice_length_supported(int M);
 // threads per slice and slices per block the slice kernel uses for M
@@ -132,6 +162,7 @@ cudaError_t noalloc_scratch(void **ptr);
 
 // One segment of twiddle table: count entries at base + offset.  ns == 0:
 // entry i = w_N^i.  ns > 0: entry r * ns + k = w_N^{k r} (a slice-pass table).
+// ns == -1: the fp16 DFT-64 operand (count = 4096 eight-byte slots).
 struct TableSeg {
     long long offset;
     long long count;
@@ -140,7 +171,7 @@ struct TableSeg {
 };
 struct TableSegs {
     int n;
-    TableSeg seg[1 + 2 * kMaxPasses];
+    TableSeg seg[3 + 2 * kMaxPasses];
 };
 cudaError_t launch_make_tables(float2 *base, const TableSegs &segs, cudaStream_t s);
 

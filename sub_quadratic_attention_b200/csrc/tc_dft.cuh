@@ -1,15 +1,10 @@
-// tc_dft.cuh -- a 16-point DFT on the 5th-generation tensor cores (tcgen05).
-//
-// Each of up to 128 rows of an fp16 operand tile A holds one length-16 complex
-// input vector, K = 32 values interleaved as (re, im) of inputs 0..15.  The
-// constant operand B is the DFT matrix w16^{sr} / 16 written as a real
-// 32 x 32 matrix, so D = A B^T gives, per row, (re, im) of the 16 outputs in
-// fp32 in tensor memory:
-//   B[2s][2r] = Fr, B[2s][2r+1] = -Fi, B[2s+1][2r] = Fi, B[2s+1][2r+1] = Fr,
-//   F = w16^{s r} / 16 (the 1/16 keeps every stage within fp16 range).
-// Both tiles use the K-major, no-swizzle canonical layout: 8-row x 16-byte
-// core matrices of 128 contiguous bytes, consecutive K chunks LBO = 128 bytes
-// apart, consecutive 8-row groups SBO = 512 bytes apart.
+// tc_dft.cuh -- tcgen05 (5th-generation tensor core) building blocks of the
+// tensor-core slice pass: shared-memory matrix descriptors for the K-major,
+// no-swizzle canonical layout (8-row x 16-byte core matrices of 128
+// contiguous bytes; lbo = bytes between K-adjacent core matrices, sbo = bytes
+// between 8-row groups), the kind::f16 instruction descriptor, MMA issue and
+// commit, bounded mbarrier waits, and tensor-memory allocation, loads and
+// stores.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -19,45 +14,36 @@
 namespace spectre {
 namespace tc {
 
-constexpr uint32_t kLBO = 128;   // bytes between the 8-element K chunks
-constexpr uint32_t kSBO = 512;   // bytes between 8-row groups (4 K chunks)
-constexpr uint32_t kRowTile = 128 * 64;  // bytes of one 128-row, K = 32 tile
-
-// byte offset of element (row, k) in a K = 32 canonical tile
-__device__ __forceinline__ uint32_t tile_offset(uint32_t row, uint32_t k) {
-    return (row >> 3) * kSBO + (k >> 3) * kLBO + (row & 7) * 16 + (k & 7) * 2;
-}
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// shared-memory matrix descriptor: K-major, no swizzle, version 1
-__device__ __forceinline__ uint64_t make_desc(uint32_t saddr) {
+// shared-memory matrix descriptor: K-major, no swizzle, version 1, with the
+// byte distance lbo between K-adjacent core matrices and sbo between
+// 8-row groups (both multiples of 16)
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-    d |= (uint64_t)((kLBO >> 4) & 0x3FFF) << 16;
-    d |= (uint64_t)((kSBO >> 4) & 0x3FFF) << 32;
-    d |= (uint64_t)1 << 46;           // descriptor version for sm_100
-    return d;                          // base offset 0, layout SWIZZLE_NONE
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
 }
 
-// instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major,
-// N = 32, M = 128
-constexpr uint32_t kIdesc = (1u << 4)            // D format f32
-                          | (0u << 7)            // A format f16
-                          | (0u << 10)           // B format f16
-                          | ((32u >> 3) << 17)   // N >> 3
-                          | ((128u >> 4) << 24); // M >> 4
+// instruction descriptor: kind::f16 with fp16 A and B (both K-major), fp32 D,
+// M = 128 rows and n columns (n a multiple of 16 in [16, 256])
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t n) {
+    return (1u << 4) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t accumulate) {
+                                        uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
-        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -102,17 +88,54 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase, uint32_
     return false;
 }
 
-// one warp allocates ncols columns of tensor memory; the base lands in *slot
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+__device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(base), "r"(ncols)
+                 : "memory");
+}
+
+// allocation without giving up the permit (a block that allocates twice
+// relinquishes after its last allocation)
+__device__ __forceinline__ void tmem_alloc_keep(uint32_t *slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :
                  : "r"(smem_u32(slot)), "r"(ncols)
                  : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(base), "r"(ncols)
-                 : "memory");
+
+// 16 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
+
+// store 16 fp32 values to consecutive columns of this thread's TMEM lane and
+// wait for the store
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        :
+        : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+          "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+          "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+          "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+          "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane
@@ -132,54 +155,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
-}
-
-// Fill the 32 x 32 fp16 DFT16/16 operand (2 KB) in canonical layout; all
-// threads of the block participate.  w16^e = cos(pi e / 8) - i sin(pi e / 8)
-// comes from cos(pi m / 8), m = 0..4, by symmetry.
-__device__ __forceinline__ float cos_pi8(int m) {  // cos(pi m / 8), m in [0, 16)
-    const float c[5] = {1.0f, 0.92387953251128674f, 0.70710678118654752f,
-                        0.38268343236508977f, 0.0f};
-    m &= 15;
-    if (m > 8) m = 16 - m;             // cos is even about pi
-    return m <= 4 ? c[m] : -c[8 - m];  // cos(pi - x) = -cos(x)
-}
-__device__ __forceinline__ void fill_dft16_operand(unsigned char *b_tile) {
-    for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) {
-        const int n = i >> 5, k = i & 31;
-        const int e = ((n >> 1) * (k >> 1)) & 15;
-        const float cs = cos_pi8(e), sn = cos_pi8(e - 4);   // sin x = cos(x - pi/2)
-        const float fr = cs * 0.0625f, fi = -sn * 0.0625f;
-        float val;
-        if ((n & 1) == 0)
-            val = (k & 1) == 0 ? fr : -fi;
-        else
-            val = (k & 1) == 0 ? fi : fr;
-        *reinterpret_cast<__half *>(b_tile + tile_offset(n, k)) = __float2half_rn(val);
-    }
-}
-
-// Store this thread's 16 complex values (times s when SCALED) as row `row`
-// of an A tile.
-template <bool SCALED>
-__device__ __forceinline__ void put_row(unsigned char *a_tile, uint32_t row, const float2 (&v)[16],
-                                        float s) {
-    auto h = [&](float2 x) {
-        return SCALED ? __floats2half2_rn(x.x * s, x.y * s) : __floats2half2_rn(x.x, x.y);
-    };
-#pragma unroll
-    for (int c = 0; c < 4; c++) {
-        __half2 h0 = h(v[4 * c]);
-        __half2 h1 = h(v[4 * c + 1]);
-        __half2 h2 = h(v[4 * c + 2]);
-        __half2 h3 = h(v[4 * c + 3]);
-        uint4 u;
-        u.x = *reinterpret_cast<uint32_t *>(&h0);
-        u.y = *reinterpret_cast<uint32_t *>(&h1);
-        u.z = *reinterpret_cast<uint32_t *>(&h2);
-        u.w = *reinterpret_cast<uint32_t *>(&h3);
-        *reinterpret_cast<uint4 *>(a_tile + tile_offset(row, 8 * c)) = u;
-    }
 }
 
 }  // namespace tc

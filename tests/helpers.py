@@ -18,8 +18,9 @@ def to_device(inputs):
     return {k: v.cuda() for k, v in inputs.items()}
 
 
-def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=False):
-    """Run the CUDA path through the C ABI.  Returns (out_f32 or None, y) on CPU."""
+def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None):
+    """Run the CUDA path through the C ABI.  Returns (out_f32 or None, y) on CPU.
+    tensor_cores: None keeps the plan's default slice pass, True/False sets it."""
     from sub_quadratic_attention_b200 import binding
     from sub_quadratic_attention_b200.binding import SpectreMix
 

@@ -58,16 +58,51 @@ def test_shape_sweep_bf16(B, L, H, D, F):
     check_parity(w, out, y, out_ref, y_ref)
 
 
-@pytest.mark.parametrize("case", ["bf16_long", (1, 65536, 2, 8, 8192), (2, 65536, 3, 5, 32769)])
+def _expected_slice_pass(w):
+    """The documented range of the tensor-core slice pass: bf16 I/O, L = 65536
+    (R = 16, M = 4096 = 64 x 64), and no slice f1 with more than two live k2
+    groups, group g covering bins f = f1 + 16 (k1 + 64 k2), k2 in [8g, 8g + 8)."""
+    if w.dtype != "bf16" or w.L != 65536:
+        return "cuda_cores"
+    R = 16
+
+    def live(g, f1):
+        return f1 + R * 512 * g < w.F or f1 + R * (63 + 64 * (8 * g + 7)) > w.L - w.F
+
+    worst = max(sum(live(g, f1) for g in range(8)) for f1 in range(R // 2 + 1))
+    return "tensor_cores" if worst <= 2 else "cuda_cores"
+
+
+@pytest.mark.parametrize("case", ["bf16_long", (1, 65536, 2, 8, 8192), (2, 65536, 3, 5, 1000),
+                                  (1, 65536, 3, 5, 1), (1, 65536, 1, 64, 4000),
+                                  (2, 65536, 3, 5, 32769)])
 def test_tensor_core_variant(case):
-    """The slice pass with its length-16 DFT stages on the tensor cores
-    (fp16 operands, fp32 accumulation) meets the bf16 bar as well."""
+    """The slice pass on the tensor cores (two DFT-64 MMA passes per 4096-point
+    transform, fp16 operands, fp32 accumulation) meets the bf16 bar as well:
+    odd channel counts (a dead half block), F = 1 (slices with no live bin),
+    and a shape outside its range (no truncation) that keeps the CUDA-core
+    slice pass."""
+    from sub_quadratic_attention_b200.binding import SpectreMix
+
     w = WORKLOADS[case] if isinstance(case, str) else custom(*case, dtype="bf16")
+    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps, tensor_cores=True) as mix:
+        assert mix.slice_pass == _expected_slice_pass(w)
     inp = make_inputs(w)
     out, y = run_library(w, inp, tensor_cores=True)
     out_ref, y_ref = oracle_full(w, inp)
     e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
     print(f"tensor cores {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+@pytest.mark.parametrize("name", ["bf16_long", "bf16_mixed_radix"])
+def test_cuda_core_slice_pass_bf16(name):
+    """The CUDA-core slice pass (the option switched off) on the bf16 workloads."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    out, y = run_library(w, inp, tensor_cores=False)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"cuda cores {name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
 
 
 def test_zero_gate_gives_layernorm_of_x():
