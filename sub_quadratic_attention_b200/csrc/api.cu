@@ -200,8 +200,10 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     if (W == C && C >= 256) g->chunk = (int)align_up((size_t)(C + 3) / 4, 64);
     const size_t slices = (size_t)B * C * NF;
     g->a_bytes = align_up((size_t)3 * B * W * NF * M * sizeof(float2), 256);
-    g->p_bytes = align_up(slices * M * (g->p16 ? 4 : 8), 256);
-    g->s_bytes = align_up(slices * sizeof(float), 256) + 256;   // scales, then the error word
+    // fp16 P interleaves channel pairs: 2 ceil(C / 2) channel lanes
+    const size_t pslices = g->p16 ? (size_t)B * 2 * ((C + 1) / 2) * NF : slices;
+    g->p_bytes = align_up(pslices * M * (g->p16 ? 4 : 8), 256);
+    g->s_bytes = align_up(pslices * sizeof(float), 256) + 256;   // scales, then the error word
     return SPECTRE_OK;
 }
 
@@ -291,6 +293,7 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     ia.T2C = g.T2C; ia.ZS = g.ZS; ia.eps = g.eps;
     ia.reg_variant = g.inv_reg;
     ia.vec2 = (g.C % 2 == 0) ? 1 : 0;
+    ia.nsm = g.nsm;
     e = mark(s);
     if (e == cudaSuccess) e = launch_rows_inv_ln(g.R, g.dtype, ia, s);
     if (e == cudaSuccess) e = mark(s);

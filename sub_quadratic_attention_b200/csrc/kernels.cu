@@ -245,7 +245,7 @@ __device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bo
 // as fp16 (round to nearest); pscale receives 1/s.  Otherwise fp32.  smax is
 // this slice's shared max word, zeroed at kernel start.
 struct PStore {
-    void *dst;        // slice base (float2 * or __half2 *)
+    void *dst;        // slice base (float2 *, or __half2 * at the channel's lane of its pair)
     float *pscale;    // this slice's scale slot
     int *smax;
     bool live, p16;
@@ -265,7 +265,7 @@ __device__ __forceinline__ float slice_scale(PStore &ps, float local_max) {
 __device__ __forceinline__ void pstore(const PStore &ps, int t2, float2 v, float s) {
     if (!ps.live) return;
     if (ps.p16)
-        static_cast<__half2 *>(ps.dst)[t2] = __floats2half2_rn(v.x * s, v.y * s);
+        static_cast<__half2 *>(ps.dst)[2 * t2] = __floats2half2_rn(v.x * s, v.y * s);
     else
         static_cast<float2 *>(ps.dst)[t2] = v;
 }
@@ -368,11 +368,16 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     const int h = c / a.D;
     const size_t sig_stride = (size_t)a.B * a.Cw * NF * M;
     const float2 *srcA = a.A + (size_t)bcl * NF * M + (size_t)f1 * M;
-    const size_t pslice = ((size_t)b * a.C + c) * NF + f1;
     PStore ps;
-    ps.dst = a.p16 ? static_cast<void *>(static_cast<__half2 *>(a.P) + pslice * M)
-                   : static_cast<void *>(static_cast<float2 *>(a.P) + pslice * M);
-    ps.pscale = a.pscale + pslice;
+    if (a.p16) {
+        const size_t pslice = p16_pair_slice(b, c, f1, a.C, NF);
+        ps.dst = static_cast<__half2 *>(a.P) + 2 * pslice * M + (c & 1);
+        ps.pscale = a.pscale + 2 * pslice + (c & 1);
+    } else {
+        const size_t pslice = ((size_t)b * a.C + c) * NF + f1;
+        ps.dst = static_cast<float2 *>(a.P) + pslice * M;
+        ps.pscale = nullptr;
+    }
     ps.smax = &smax[sl];
     ps.live = live;
     ps.p16 = a.p16 != 0;
@@ -438,30 +443,35 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
         if (t2 >= a.M) continue;
         const int c0 = 2 * cp;
         const bool has1 = c0 + 1 < a.C;
-        const size_t sa = ((size_t)b * a.C + c0) * NF;
+        // fp32 P: slices (c0, f1) and (c0 + 1, f1); fp16 P: the pair's slice
+        const size_t sa = P16 ? p16_pair_slice(b, c0, 0, a.C, NF) : ((size_t)b * a.C + c0) * NF;
         const size_t sb = sa + NF;
-        auto ld = [&](size_t slice, bool ok) -> float2 {
-            if (!ok) return make_float2(0.f, 0.f);
+        auto ld2 = [&](int f1, float2 &pa, float2 &pb) {
             if constexpr (P16) {
-                float2 v = __half22float2(__ldg(static_cast<const __half2 *>(a.P) + slice * a.M + t2));
-                return cscale(v, __ldg(a.pscale + slice));
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(a.P) + (sa + f1) * a.M + t2);
+                const float2 sc = __ldg(reinterpret_cast<const float2 *>(a.pscale) + sa + f1);
+                pa = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.x)), sc.x);
+                pb = has1 ? cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.y)), sc.y)
+                          : make_float2(0.f, 0.f);
             } else {
-                return __ldg(static_cast<const float2 *>(a.P) + slice * a.M + t2);
+                pa = __ldg(static_cast<const float2 *>(a.P) + (sa + f1) * a.M + t2);
+                pb = has1 ? __ldg(static_cast<const float2 *>(a.P) + (sb + f1) * a.M + t2)
+                          : make_float2(0.f, 0.f);
             }
         };
         float2 Z[R];
         {
-            float2 a0 = ld(sa, true), aN = ld(sa + R / 2, true);
-            float2 b0 = ld(sb, has1);
-            float2 bN = ld(sb + R / 2, has1);
+            float2 a0, aN, b0, bN;
+            ld2(0, a0, b0);
+            ld2(R / 2, aN, bN);
             // DC and Nyquist: imaginary parts dropped; conj() for the inverse
             Z[0] = make_float2(a0.x, -b0.x);
             Z[R / 2] = make_float2(aN.x, -bN.x);
         }
 #pragma unroll
         for (int f1 = 1; f1 < R / 2; f1++) {
-            float2 pv = ld(sa + f1, true);
-            float2 qv = ld(sb + f1, has1);
+            float2 pv, qv;
+            ld2(f1, pv, qv);
             // Z[f1] = P_a + i P_b ; Z[R - f1] = conj(P_a) + i conj(P_b); stored conjugated
             Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
             Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
@@ -567,25 +577,35 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     float z0[R], z1[R];
     {
         float2 Z[R];
-        const size_t sa = ((size_t)b * a.C + c0) * NF;       // slice index of (c0, f1 = 0)
-        const size_t sb = sa + NF;
-        auto ld = [&](size_t slice, bool ok) -> float2 {
-            if (!ok) return make_float2(0.f, 0.f);
+        // fp32 P: slices (c0, f1) and (c0 + 1, f1); fp16 P: the pair's slice,
+        // one 8-byte load for both channels
+        const int cc = live ? c0 : 0, tt = live ? t2 : 0;
+        const size_t sa = P16 ? p16_pair_slice(b, cc, 0, a.C, NF) : ((size_t)b * a.C + cc) * NF;
+        const size_t pofs = sa * a.M + tt;
+        const int fstride = a.M, cstride = NF * a.M;
+        auto ld2 = [&](int f1, float2 &pa, float2 &pb) {
+            pa = pb = make_float2(0.f, 0.f);
+            if (!live) return;
             if constexpr (P16) {
-                float2 v = __half22float2(__ldg(static_cast<const __half2 *>(a.P) + slice * a.M + t2));
-                return cscale(v, __ldg(a.pscale + slice));
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(a.P) + pofs + f1 * fstride);
+                const float2 sc = __ldg(reinterpret_cast<const float2 *>(a.pscale) + sa + f1);
+                pa = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.x)), sc.x);
+                if (has1) pb = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.y)), sc.y);
             } else {
-                return __ldg(static_cast<const float2 *>(a.P) + slice * a.M + t2);
+                const float2 *p = static_cast<const float2 *>(a.P) + pofs;
+                pa = __ldg(p + f1 * fstride);
+                if (has1) pb = __ldg(p + cstride + f1 * fstride);
             }
         };
-        float2 a0 = ld(sa, live), aN = ld(sa + R / 2, live);
-        float2 b0 = ld(sb, has1), bN = ld(sb + R / 2, has1);
+        float2 a0, aN, b0, bN;
+        ld2(0, a0, b0);
+        ld2(R / 2, aN, bN);
         Z[0] = make_float2(a0.x, -b0.x);
         Z[R / 2] = make_float2(aN.x, -bN.x);
 #pragma unroll
         for (int f1 = 1; f1 < R / 2; f1++) {
-            float2 pv = ld(sa + f1, live);
-            float2 qv = ld(sb + f1, has1);
+            float2 pv, qv;
+            ld2(f1, pv, qv);
             Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
             Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
         }
@@ -597,9 +617,9 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
         }
     }
     const T *x = static_cast<const T *>(a.x);
-    const size_t tok0 = (size_t)b * a.L + t2;
-    const size_t rowstep = (size_t)a.M * a.C;
-    const T *xp = x + tok0 * a.C + c0;
+    const size_t tok0 = (size_t)b * a.L + (live ? t2 : 0);
+    const int rowstep = a.M * a.C;                      // elements between t1 rows
+    const T *xp = x + tok0 * a.C + (live ? c0 : 0);
     float s[R];
 #pragma unroll
     for (int t1 = 0; t1 < R; t1++) {
@@ -624,7 +644,7 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     }
     const float invC = 1.0f / (float)a.C;
     // two reductions over the channels of each row: sum(z), then sum((z - mean)^2);
-    // stat[0][.] holds the means, stat[1][.] the variances
+    // stat[0][.] holds the means, stat[1][.] the reciprocal standard deviations
 #pragma unroll 1
     for (int pass = 0; pass < 2; pass++) {
         if (pass == 1) {
@@ -646,11 +666,14 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
             HalvingReduce<R, B0, 5>::run(v, lane, row0);
 #pragma unroll
             for (int i = 0; i < NOUT; i++) part[(warp * T2C + tl) * R + row0 + i] = v[i];
-        }        __syncthreads();
-        for (int i = tid; i < T2C * R; i += nthr) {
-            float acc = 0.f;
-            for (int w = 0; w < nwarps; w++) acc += part[w * T2C * R + i];
-            stat[pass * T2C * R + i] = acc * invC;
+        }
+        __syncthreads();
+        // a warp per row sums the row's per-warp partials (lane w: warp w's,
+        // w < nwarps <= 32), in a fixed order
+        for (int i = warp; i < T2C * R; i += nwarps) {
+            float acc = lane < nwarps ? part[lane * T2C * R + i] : 0.f;
+            acc = warp_sum(acc) * invC;
+            if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
         }
         __syncthreads();
     }
@@ -661,7 +684,7 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
 #pragma unroll
     for (int t1 = 0; t1 < R; t1++) {
         const float mu = stat[tl * R + t1];
-        const float rstd = rsqrtf(stat[T2C * R + tl * R + t1] + a.eps);
+        const float rstd = stat[T2C * R + tl * R + t1];
         const float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
         const float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
         if (has1 && a.vec2) {
@@ -671,6 +694,174 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
             if (has1) Elem<T>::store(yp + t1 * rowstep + 1, y1);
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// inverse row pass + residual + LayerNorm, prefetching variant (R = 16,
+// bf16 I/O with fp16 P, C a multiple of 8, C <= 512).  A persistent block of
+// 2 x CP threads (thread = tl + 2 cp: one of two token columns t2, one channel
+// pair) walks pairs of columns; while it inverts and normalises one pair from
+// a shared-memory stage, cp.async copies the next pair's P (per channel pair
+// and f1, both columns' two fp16 complex values: 16 contiguous bytes) and its
+// 2 x 16 rows of x into the other stage, so no register holds data in
+// flight.  The x rows are padded by 32 values so the two columns' rows fall
+// on different banks.  The arithmetic per column is that of
+// spectre_rows_inv_ln_reg with T2C = 2.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :
+                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+constexpr int kInvPipeMaxC = 512;
+
+// shared-memory words of one stage: P [NF][CP][2 columns] as uint2 (the pair's
+// two half2), then x [16 rows][2 columns][C + 32] bf16
+__host__ __device__ inline int inv_pipe_stage_words(int C) {
+    return 9 * (C / 2) * 2 * 2 + 16 * 2 * (C + 32) / 2;
+}
+
+template <bool DEBUG_OUT>
+__global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(RowsInvArgs a) {
+    constexpr int R = 16, NF = R / 2 + 1, T2C = 2;
+    extern __shared__ float4 smem_f4[];
+    const int C = a.C, CP = C / 2, XS = C + 32;
+    const int nthr = blockDim.x, nwarps = nthr >> 5;
+    const int stage_words = inv_pipe_stage_words(C);
+    uint32_t *stage0 = reinterpret_cast<uint32_t *>(smem_f4);
+    float *part = reinterpret_cast<float *>(stage0 + 2 * stage_words);   // [nwarps][T2C][R]
+    float *stat = part + nwarps * T2C * R;                               // [2][T2C][R]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tl = tid & 1, cp = tid >> 1, c0 = 2 * cp;
+    const bool live = cp < CP;
+    const int npair_cols = a.M / T2C;
+    const long long ngroups = (long long)a.B * npair_cols;
+    const uint4 *P4 = static_cast<const uint4 *>(a.P);       // one uint4 = 2 columns of a pair
+    const float2 *ps2 = reinterpret_cast<const float2 *>(a.pscale);
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
+    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
+    const int rowstep = a.M * C;
+
+    auto prefetch = [&](long long grp, int st) {
+        const int b = (int)(grp / npair_cols), t2 = (int)(grp % npair_cols) * T2C;
+        uint32_t *pst = stage0 + st * stage_words;
+        uint32_t *xst = pst + NF * CP * 4;
+        for (int i = tid; i < NF * CP; i += nthr) {            // i = f1 * CP + pair
+            const int f1 = i / CP, pr = i - f1 * CP;
+            const size_t slice = ((size_t)b * CP + pr) * NF + f1;
+            cp_async16(pst + 4 * i, P4 + (slice * a.M + t2) / 2);
+        }
+        const __nv_bfloat16 *xb = x + ((size_t)b * a.L + t2) * C;
+        const int chunks = C / 8;                              // 16-byte pieces per row
+        for (int i = tid; i < R * T2C * chunks; i += nthr) {   // i = (t1 * 2 + col) * chunks + k
+            const int rowi = i / chunks, k = i - rowi * chunks;
+            const int t1 = rowi >> 1, col = rowi & 1;
+            cp_async16(xst + rowi * (XS / 2) + 4 * k, xb + (size_t)t1 * rowstep + (size_t)col * C + 8 * k);
+        }
+    };
+
+    const float g0 = live ? __ldg(a.gamma + c0) : 0.f, be0 = live ? __ldg(a.beta + c0) : 0.f;
+    const float g1 = live ? __ldg(a.gamma + c0 + 1) : 0.f, be1 = live ? __ldg(a.beta + c0 + 1) : 0.f;
+    const float invC = 1.0f / (float)C;
+    long long grp = blockIdx.x;
+    if (grp < ngroups) prefetch(grp, 0);
+    cp_async_commit();
+#pragma unroll 1
+    for (int k = 0; grp < ngroups; k++, grp += gridDim.x) {
+        const long long nxt = grp + gridDim.x;
+        if (nxt < ngroups) prefetch(nxt, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        const uint32_t *pst = stage0 + (k & 1) * stage_words;
+        const uint32_t *xst = pst + NF * CP * 4;
+        const int b = (int)(grp / npair_cols), t2 = (int)(grp % npair_cols) * T2C + tl;
+        float z0[R], z1[R], s[R];
+        {
+            float2 Z[R];
+            const size_t sa = ((size_t)b * CP + (live ? cp : 0)) * NF;
+            auto ld2 = [&](int f1, float2 &pa, float2 &pb) {
+                pa = pb = make_float2(0.f, 0.f);
+                if (!live) return;
+                const uint2 u = reinterpret_cast<const uint2 *>(pst)[(f1 * CP + cp) * 2 + tl];
+                const float2 sc = __ldg(ps2 + sa + f1);
+                pa = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.x)), sc.x);
+                pb = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.y)), sc.y);
+            };
+            float2 a0, aN, b0, bN;
+            ld2(0, a0, b0);
+            ld2(R / 2, aN, bN);
+            Z[0] = make_float2(a0.x, -b0.x);
+            Z[R / 2] = make_float2(aN.x, -bN.x);
+#pragma unroll
+            for (int f1 = 1; f1 < R / 2; f1++) {
+                float2 pv, qv;
+                ld2(f1, pv, qv);
+                Z[f1] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
+                Z[R - f1] = make_float2(pv.x + qv.y, pv.y - qv.x);
+            }
+            Dft<R>::run(Z);
+            const size_t tok0 = (size_t)b * a.L + t2;
+#pragma unroll
+            for (int t1 = 0; t1 < R; t1++) {
+                z0[t1] = Z[t1].x;
+                z1[t1] = -Z[t1].y;
+                if (DEBUG_OUT && live)
+                    *reinterpret_cast<float2 *>(a.out_f32 + (tok0 + (size_t)t1 * a.M) * C + c0) =
+                        make_float2(z0[t1], z1[t1]);
+                const uint32_t xw = live ? xst[(t1 * 2 + tl) * (XS / 2) + cp] : 0u;
+                const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw));
+                z0[t1] = live ? z0[t1] + xv.x : 0.f;
+                z1[t1] = live ? z1[t1] + xv.y : 0.f;
+                s[t1] = z0[t1] + z1[t1];
+            }
+        }
+        // LayerNorm statistics of the 2 x R token rows, two passes
+#pragma unroll 1
+        for (int pass = 0; pass < 2; pass++) {
+            if (pass == 1) {
+#pragma unroll
+                for (int t1 = 0; t1 < R; t1++) {
+                    const float mu = stat[tl * R + t1];
+                    const float d0 = z0[t1] - mu, d1 = z1[t1] - mu;
+                    s[t1] = live ? fmaf(d0, d0, d1 * d1) : 0.f;
+                }
+            }
+            {
+                // channel pairs of one column differ in lane bits [1, 5)
+                float v[R];
+#pragma unroll
+                for (int t1 = 0; t1 < R; t1++) v[t1] = s[t1];
+                int row0 = 0;
+                HalvingReduce<R, 1, 5>::run(v, lane, row0);
+                part[(warp * T2C + tl) * R + row0] = v[0];
+            }
+            __syncthreads();
+            for (int i = warp; i < T2C * R; i += nwarps) {
+                float acc = lane < nwarps ? part[lane * T2C * R + i] : 0.f;
+                acc = warp_sum(acc) * invC;
+                if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
+            }
+            __syncthreads();
+        }
+        if (live) {
+            __nv_bfloat16 *yp = y + ((size_t)b * a.L + t2) * C + c0;
+#pragma unroll
+            for (int t1 = 0; t1 < R; t1++) {
+                const float mu = stat[tl * R + t1], rstd = stat[T2C * R + tl * R + t1];
+                Elem<__nv_bfloat16>::store2(yp + t1 * rowstep, fmaf((z0[t1] - mu) * rstd, g0, be0),
+                                            fmaf((z1[t1] - mu) * rstd, g1, be1));
+            }
+        }
+        // every read of this stage and of stat is done before the stage is refilled
+        __syncthreads();
+    }
+    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------
@@ -752,6 +943,22 @@ void slice_geometry(int M, int *nt, int *spb, size_t *smem) {
 
 template <int R, typename T>
 static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
+    if constexpr (R == 16 && std::is_same<T, __nv_bfloat16>::value) {
+        if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0) {
+            const int threads = ((a.C + 31) / 32) * 32;         // 2 columns x C / 2 pairs
+            const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32) * 32 + 64) * 4;
+            auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true> : spectre_rows_inv_ln_pipe<false>;
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess ||
+                per_sm < 1)
+                per_sm = 1;
+            const long long ngroups = (long long)a.B * (a.M / 2);
+            const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
+            k<<<(unsigned)(ngroups < cap ? ngroups : cap), threads, smem, s>>>(a);
+            return cudaGetLastError();
+        }
+    }
     if constexpr (R <= 16) if (a.reg_variant) {
         dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
         const int CP = (a.C + 1) / 2;

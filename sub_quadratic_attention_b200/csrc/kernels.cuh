@@ -40,10 +40,18 @@ struct RowsFwdArgs {
     int vec2;             // C even: load channel pairs as one vector
 };
 
+// fp16 P (bf16 I/O) interleaves the two channels c = 2 cp, 2 cp + 1 of a pair:
+// the half2 of (b, c, f1, t2) is number 2 (pslice M + t2) + (c & 1), and its
+// scale pscale[2 pslice + (c & 1)], with pslice = (b CP + cp) NF + f1,
+// CP = ceil(C / 2), NF = R / 2 + 1.  fp32 P (fp32 I/O) is [B][C][NF][M].
+__host__ __device__ inline size_t p16_pair_slice(int b, int c, int f1, int C, int NF) {
+    return ((size_t)b * ((C + 1) / 2) + c / 2) * NF + f1;
+}
+
 struct SliceArgs {
     const float2 *A;      // [3][B][Cw][R/2+1][M]: the wave's channels
-    void *P;              // [B][C][R/2+1][M]: float2, or __half2 scaled by 1/pscale
-    float *pscale;        // [B][C][R/2+1]: P = stored * pscale (p16 only)
+    void *P;              // float2 [B][C][NF][M], or __half2 pair-interleaved (p16_pair_slice)
+    float *pscale;        // p16: P = stored * pscale, pair-interleaved like P
     const float2 *twL;
     const float *G;       // [H][L/2+1]
     SliceTables tabs;
@@ -61,7 +69,7 @@ struct SliceArgs {
 };
 
 struct RowsInvArgs {
-    const void *P;        // float2 (fp32 I/O) or __half2 (bf16 I/O) with pscale
+    const void *P;        // float2 [B][C][NF][M] (fp32 I/O) or pair-interleaved __half2 with pscale
     const float *pscale;
     const void *x;
     const float *gamma, *beta;
@@ -71,6 +79,7 @@ struct RowsInvArgs {
     int T2C, ZS;          // t2 values per block, padded row stride of the z buffer
     int reg_variant;      // 1: register-resident LayerNorm (R <= 16, C <= 2048)
     int vec2;             // C even: channel pairs as one vector
+    int nsm;              // multiprocessors (grid of the persistent variant)
     float eps;
 };
 

@@ -254,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
         }
         if (gmask == 0) {   // every gate of the slice is zero: P = 0
             if (live) {
-                const size_t pslice = ((size_t)b * a.C + c) * NF + f1;
-                uint32_t *dst = static_cast<uint32_t *>(a.P) + pslice * kM;
-                for (int m2 = 32 * half; m2 < 32 * half + 32; m2++) dst[row + 64 * m2] = 0u;
-                if (lead) a.pscale[pslice] = 1.0f;
+                const size_t pslice = p16_pair_slice(b, c, f1, a.C, NF);
+                uint32_t *dst = static_cast<uint32_t *>(a.P) + 2 * pslice * kM + (c & 1);
+                for (int m2 = 32 * half; m2 < 32 * half + 32; m2++) dst[2 * (row + 64 * m2)] = 0u;
+                if (lead) a.pscale[2 * pslice + (c & 1)] = 1.0f;
             }
             continue;
         }
@@ -376,8 +376,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
         // P[t2] = conj(U[t2] w_L^{f1 t2}) at t2 = row + 64 m2; the scale
         // gathers 4096 / s of each transform: 2^(48 - sum of shifts)
         {
-            const size_t pslice = ((size_t)b * a.C + (live ? c : 0)) * NF + f1;
-            uint32_t *dst = static_cast<uint32_t *>(a.P) + pslice * kM;
+            const int cc = live ? c : 0;
+            const size_t pslice = p16_pair_slice(b, cc, f1, a.C, NF);
+            uint32_t *dst = static_cast<uint32_t *>(a.P) + 2 * pslice * kM + (cc & 1);
             // w_L^{f1 t2} by recurrences in m2 (step w_L^{64 f1}) from
             // w_L^{f1 (row + 1024 q)}
             const float2 step = __ldg(a.twL + 64 * f1);
@@ -389,11 +390,12 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
 #pragma unroll
                 for (int i = 0; i < 16; i++) {
                     const float2 u = cmul(make_float2(d[2 * i], d[2 * i + 1]), t);
-                    if (live) dst[row + 64 * (16 * q + i)] = h2_bits(u.x, -u.y);
+                    if (live) dst[2 * (row + 64 * (16 * q + i))] = h2_bits(u.x, -u.y);
                     t = cmul(t, step);
                 }
             }
-            if (live && lead) a.pscale[pslice] = ldexpf(1.0f, 48 - shift_sum);
+            if (live && lead)
+                a.pscale[2 * pslice + (cc & 1)] = ldexpf(1.0f, min(127, 48 - shift_sum));
         }
     }
     if (abort && tid == 0 && a.err) atomicOr(a.err, 1);
