@@ -259,6 +259,7 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
             fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
             fa.c_lo = c_lo; fa.Cw = Cw;
             fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
+            fa.nsm = g.nsm;
             e = mark(st);
             if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, st);
             if (e != cudaSuccess) return cuda_status(e);

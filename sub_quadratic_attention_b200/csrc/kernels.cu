@@ -121,6 +121,114 @@ __global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwd
 }
 
 // ---------------------------------------------------------------------------
+// row pass, prefetching variant (R = 16, bf16 inputs, channel chunks that are
+// multiples of 64).  Work items are (tile, signal) with tiles of 8 t2 x 64
+// channels; a persistent block computes one item from a shared-memory stage
+// while cp.async copies the next item's 16 x 8 row segments (64 bf16 each)
+// into the other stage.  Rows are padded to 80 values so the warp's 4 t2 x 8
+// channel-pair reads fall on 32 different banks.  Thread mapping, arithmetic
+// and stores are those of spectre_rows_fwd.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :
+                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async16_rows(void *smem_dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :
+                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
+                 : "memory");
+}
+
+constexpr int kFwdPipeRow = 80;                          // bf16 per padded row
+constexpr int kFwdPipeStage = 16 * 8 * kFwdPipeRow / 2;  // 4-byte words per stage
+
+__global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
+    constexpr int R = 16, NF = R / 2 + 1;
+    extern __shared__ float4 smem_f4[];
+    uint32_t *stage0 = reinterpret_cast<uint32_t *>(smem_f4);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t2l = (warp & 1) * 4 + (lane & 3);           // 0..7
+    const int cpl = (warp >> 1) * 8 + (lane >> 2);         // 0..31
+    const int ntg = a.M / 8, ncg = a.Cw / 64;
+    const long long nitems = 3LL * ntg * ncg * a.B;
+    const size_t rowstep = (size_t)a.M * a.C;
+    const size_t plane = (size_t)a.B * a.Cw * NF * a.M;
+
+    // item = ((b * ncg + cg) * ntg + tg) * 3 + sig
+    auto decode = [&](long long item, int &sig, int &tg, int &cg, int &b) {
+        sig = (int)(item % 3);
+        long long r = item / 3;
+        tg = (int)(r % ntg);
+        r /= ntg;
+        cg = (int)(r % ncg);
+        b = (int)(r / ncg);
+    };
+    auto prefetch = [&](long long item, int st) {
+        int sig, tg, cg, b;
+        decode(item, sig, tg, cg, b);
+        uint32_t *dst = stage0 + st * kFwdPipeStage;
+        const void *sp = sig == 0 ? a.q : (sig == 1 ? a.k : a.v);
+        const __nv_bfloat16 *base = static_cast<const __nv_bfloat16 *>(sp) +
+                                    ((size_t)b * a.L + (size_t)tg * 8) * a.C + a.c_lo + 64 * cg;
+        for (int i = tid; i < 16 * 8 * 8; i += 256) {       // (t1, t2 row, 16-byte piece)
+            const int piece = i & 7, rr = i >> 3, t1 = rr >> 3, tr = rr & 7;
+            cp_async16_rows(dst + rr * (kFwdPipeRow / 2) + 4 * piece,
+                            base + (size_t)t1 * rowstep + (size_t)tr * a.C + 8 * piece);
+        }
+    };
+
+    long long it = blockIdx.x;
+    if (it < nitems) prefetch(it, 0);
+    cp_async_commit();
+#pragma unroll 1
+    for (int k = 0; it < nitems; k++, it += gridDim.x) {
+        const long long nxt = it + gridDim.x;
+        if (nxt < nitems) prefetch(nxt, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait1();
+        __syncthreads();
+        int sig, tg, cg, b;
+        decode(it, sig, tg, cg, b);
+        const uint32_t *stg = stage0 + (k & 1) * kFwdPipeStage;
+        const int t2 = tg * 8 + t2l;
+        const int cl = 64 * cg + 2 * cpl;                  // channel within the chunk
+        float2 z[R];
+#pragma unroll
+        for (int t1 = 0; t1 < R; t1++) {
+            const uint32_t w = stg[(t1 * 8 + t2l) * (kFwdPipeRow / 2) + cpl];
+            z[t1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
+        }
+        Dft<R>::run(z);
+        float2 *dst0 = a.A + sig * plane + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
+        float2 *dst1 = dst0 + (size_t)NF * a.M;
+#pragma unroll
+        for (int f1 = 0; f1 < NF; f1++) {
+            float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
+            float2 xa = cscale(cadd(zf, zc), 0.5f);
+            float2 d = csub(zf, zc);
+            float2 xb = make_float2(0.5f * d.y, -0.5f * d.x);
+            if (f1 > 0) {
+                float2 w = __ldg(a.twL + f1 * t2);
+                xa = cmul(xa, w);
+                xb = cmul(xb, w);
+            }
+            dst0[(size_t)f1 * a.M] = xa;
+            dst1[(size_t)f1 * a.M] = xb;
+        }
+        // every read of this stage is done before it is refilled
+        __syncthreads();
+    }
+    cp_async_wait_all();
+}
+
+// ---------------------------------------------------------------------------
 // slice pass
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int spad(int i) { return i + (i >> 4); }
@@ -708,16 +816,6 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
 // on different banks.  The arithmetic per column is that of
 // spectre_rows_inv_ln_reg with T2C = 2.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                 :
-                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 constexpr int kInvPipeMaxC = 512;
 
 // shared-memory words of one stage: P [NF][CP][2 columns] as uint2 (the pair's
@@ -869,6 +967,18 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
 // ---------------------------------------------------------------------------
 template <int R>
 static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a, cudaStream_t s) {
+    if (R == 16 && dtype == 1 && a.vec2 && a.C % 8 == 0 && a.c_lo % 64 == 0 && a.Cw % 64 == 0 &&
+        a.M % 8 == 0) {
+        const size_t smem = (size_t)2 * kFwdPipeStage * 4;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spectre_rows_fwd_pipe, 256, smem) !=
+                cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const long long nitems = 3LL * (a.M / 8) * (a.Cw / 64) * a.B;
+        const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
+        spectre_rows_fwd_pipe<<<(unsigned)(nitems < cap ? nitems : cap), 256, smem, s>>>(a);
+        return cudaGetLastError();
+    }
     dim3 grid((a.M + 7) / 8, (a.Cw + 63) / 64, a.B);
     if (dtype == 0)
         spectre_rows_fwd<R, float><<<grid, 256, 0, s>>>(a);

@@ -38,6 +38,7 @@ struct RowsFwdArgs {
     int B, L, M, C;
     int c_lo, Cw;         // channel wave (c_lo even)
     int vec2;             // C even: load channel pairs as one vector
+    int nsm;              // multiprocessors (grid of the persistent variant)
 };
 
 // fp16 P (bf16 I/O) interleaves the two channels c = 2 cp, 2 cp + 1 of a pair:
