@@ -97,16 +97,16 @@ struct Mma {
             tc::fence_after();
             if (full_n) {
                 uint32_t acc = 0;
-                for (int ks = 0; ks < 8; ks++) {
-                    if (!((ksteps >> ks) & 1u)) continue;
+                for (uint32_t km = ksteps; km; km &= km - 1) {
+                    const int ks = __ffs(km) - 1;
                     tc::mma_f16(dcol, tc::make_desc(tile + ks * 2 * kTileLBO, kTileLBO, kTileSBO),
                                 tc::make_desc(op + ks * 2 * 128, 128, 2048), tc::idesc_f16(128), acc);
                     acc = 1;
                 }
             } else {
                 uint32_t gi = 0;
-                for (int g = 0; g < 8; g++) {
-                    if (!((gmask >> g) & 1u)) continue;
+                for (uint32_t gm = gmask; gm; gm &= gm - 1) {
+                    const int g = __ffs(gm) - 1;
                     for (int ks = 0; ks < 8; ks++)
                         tc::mma_f16(dcol + 16 * gi,
                                     tc::make_desc(tile + ks * 2 * kTileLBO, kTileLBO, kTileSBO),
@@ -136,17 +136,19 @@ __device__ __forceinline__ void twiddle_transpose(uint32_t tl, const float2 *__r
                                                   unsigned char *tile, int sbase, int row, int half) {
     const float2 w1 = __ldg(twMM + 64 + row), w16 = __ldg(twMM + 16 * 64 + row);
     float2 tq = half ? cmul(w16, w16) : make_float2(1.f, 0.f);
+    // column K = 2 row of tile row sbase + 16 q + i sits at colbase + (2q + i/8) SBO + (i%8) 16
+    unsigned char *colbase = tile + tile_off(sbase, 2 * row);
 #pragma unroll 1
     for (int q = 2 * half; q < 2 * half + 2; q++) {
         float d[32];
         tc::tmem_ld32(tl + 32 * q, d);
         float2 t = tq;
         tq = cmul(tq, w16);
+        unsigned char *qb = colbase + 2 * q * kTileSBO;
 #pragma unroll
         for (int i = 0; i < 16; i++) {
             const float2 y = cmul(make_float2(d[2 * i], d[2 * i + 1]), t);
-            *reinterpret_cast<uint32_t *>(tile + tile_off(sbase + 16 * q + i, 2 * row)) =
-                h2_bits(y.x, y.y);
+            *reinterpret_cast<uint32_t *>(qb + (i >> 3) * kTileSBO + (i & 7) * 16) = h2_bits(y.x, y.y);
             t = cmul(t, w1);
         }
     }
@@ -313,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
             // the two halves take alternate groups
             uint32_t gi = 0;
 #pragma unroll 1
-            for (int g = 0; g < 8; g++) {
-                if (!((gmask >> g) & 1u)) continue;
+            for (uint32_t gm = gmask; gm; gm &= gm - 1, gi++) {
+                const int g = __ffs(gm) - 1;
                 if ((gi & 1u) == (uint32_t)half) {
                     float d[16], sv[16];
                     tc::tmem_ld16(tlD + 16 * gi, d);
@@ -339,7 +341,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
                     }
                     tc::tmem_st16(tlS + 16 * gi, sv);
                 }
-                gi++;
             }
         }
         if (abort) break;
@@ -351,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
             const float s = ldexpf(1.0f, sh);
             uint32_t gi = 0;
 #pragma unroll 1
-            for (int g = 0; g < 8; g++) {
-                if (!((gmask >> g) & 1u)) continue;
+            for (uint32_t gm = gmask; gm; gm &= gm - 1, gi++) {
+                const int g = __ffs(gm) - 1;
                 if ((gi & 1u) == (uint32_t)half) {
                     float sv[16];
                     tc::tmem_ld16(tlS + 16 * gi, sv);
@@ -366,7 +367,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
                         *reinterpret_cast<uint4 *>(tile + tile_off(trow, 16 * g + 8 * hh)) = u;
                     }
                 }
-                gi++;
             }
         }
         if (!mma.run(gmask, 0, true)) { abort = true; break; }
