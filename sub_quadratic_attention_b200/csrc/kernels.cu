@@ -671,10 +671,14 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
     constexpr bool P16 = std::is_same<T, __nv_bfloat16>::value;  // bf16 I/O: fp16 P
     extern __shared__ float4 smem_f4[];
-    float *part = reinterpret_cast<float *>(smem_f4);   // [nwarps][T2C][R], then stat[2][T2C][R]
+    // per-warp partial sums as [T2C * R rows][nwarps + 1] (the pad keeps both
+    // the per-warp writes and the per-row reads on distinct banks), then
+    // stat[2][T2C][R]
+    float *part = reinterpret_cast<float *>(smem_f4);
     const int nthr = blockDim.x;
     const int nwarps = nthr >> 5;
-    float *stat = part + nwarps * T2C * R;               // [T2C][R]
+    const int PS = nwarps + 1;
+    float *stat = part + T2C * R * PS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tl = tid & (T2C - 1), cp = tid / T2C;
     const int b = blockIdx.y;
@@ -773,13 +777,13 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
             int row0 = 0;
             HalvingReduce<R, B0, 5>::run(v, lane, row0);
 #pragma unroll
-            for (int i = 0; i < NOUT; i++) part[(warp * T2C + tl) * R + row0 + i] = v[i];
+            for (int i = 0; i < NOUT; i++) part[(tl * R + row0 + i) * PS + warp] = v[i];
         }
         __syncthreads();
         // a warp per row sums the row's per-warp partials (lane w: warp w's,
         // w < nwarps <= 32), in a fixed order
         for (int i = warp; i < T2C * R; i += nwarps) {
-            float acc = lane < nwarps ? part[lane * T2C * R + i] : 0.f;
+            float acc = lane < nwarps ? part[i * PS + lane] : 0.f;
             acc = warp_sum(acc) * invC;
             if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
         }
@@ -832,8 +836,11 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int stage_words = inv_pipe_stage_words(C);
     uint32_t *stage0 = reinterpret_cast<uint32_t *>(smem_f4);
-    float *part = reinterpret_cast<float *>(stage0 + 2 * stage_words);   // [nwarps][T2C][R]
-    float *stat = part + nwarps * T2C * R;                               // [2][T2C][R]
+    // per-warp partial sums as [T2C * R rows][nwarps + 1] (padded: distinct
+    // banks for the writes and the per-row reads), then stat[2][T2C][R]
+    const int PS = nwarps + 1;
+    float *part = reinterpret_cast<float *>(stage0 + 2 * stage_words);
+    float *stat = part + T2C * R * PS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tl = tid & 1, cp = tid >> 1, c0 = 2 * cp;
     const bool live = cp < CP;
@@ -937,11 +944,11 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
                 for (int t1 = 0; t1 < R; t1++) v[t1] = s[t1];
                 int row0 = 0;
                 HalvingReduce<R, 1, 5>::run(v, lane, row0);
-                part[(warp * T2C + tl) * R + row0] = v[0];
+                part[(tl * R + row0) * PS + warp] = v[0];
             }
             __syncthreads();
             for (int i = warp; i < T2C * R; i += nwarps) {
-                float acc = lane < nwarps ? part[lane * T2C * R + i] : 0.f;
+                float acc = lane < nwarps ? part[i * PS + lane] : 0.f;
                 acc = warp_sum(acc) * invC;
                 if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
             }
@@ -1056,7 +1063,7 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
     if constexpr (R == 16 && std::is_same<T, __nv_bfloat16>::value) {
         if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0) {
             const int threads = ((a.C + 31) / 32) * 32;         // 2 columns x C / 2 pairs
-            const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32) * 32 + 64) * 4;
+            const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32 + 1) * 32 + 64) * 4;
             auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true> : spectre_rows_inv_ln_pipe<false>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             int per_sm = 0;
@@ -1073,7 +1080,7 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
         dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
         const int CP = (a.C + 1) / 2;
         const int threads = ((a.T2C * CP + 31) / 32) * 32;
-        size_t smem = (size_t)((threads / 32) * a.T2C * R + 2 * a.T2C * R) * sizeof(float);
+        size_t smem = (size_t)((threads / 32 + 1) * a.T2C * R + 2 * a.T2C * R) * sizeof(float);
         switch (a.T2C) {
 #define SPECTRE_INV_T2C(t2c)                                                          \
     case t2c:                                                                         \
