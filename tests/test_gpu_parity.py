@@ -49,8 +49,13 @@ def test_shape_sweep_fp32(B, L, H, D, F):
 
 
 @pytest.mark.parametrize("B,L,H,D,F", [(1, 256, 1, 16, 40), (2, 12288, 2, 8, 6145),
-                                       (1, 65536, 2, 8, 8192), (1, 3072, 3, 5, 1)])
+                                       (1, 65536, 2, 8, 8192), (1, 3072, 3, 5, 1),
+                                       (1, 4096, 7, 72, 1000), (3, 4096, 4, 128, 2049)])
 def test_shape_sweep_bf16(B, L, H, D, F):
+    """bf16 shapes across the kernel variants: C = 504 (the last channel chunk
+    not a multiple of 64, so prefetching and plain row passes mix in one run;
+    dead lanes in the prefetching inverse pass) and C = 512 with B = 3 (the
+    persistent passes crossing batch boundaries)."""
     w = custom(B, L, H, D, F, dtype="bf16")
     inp = make_inputs(w)
     out, y = run_library(w, inp)
@@ -75,7 +80,7 @@ def _expected_slice_pass(w):
 
 @pytest.mark.parametrize("case", ["bf16_long", (1, 65536, 2, 8, 8192), (2, 65536, 3, 5, 1000),
                                   (1, 65536, 3, 5, 1), (1, 65536, 1, 64, 4000),
-                                  (2, 65536, 3, 5, 32769)])
+                                  (1, 65536, 7, 72, 8192), (2, 65536, 3, 5, 32769)])
 def test_tensor_core_variant(case):
     """The slice pass on the tensor cores (two DFT-64 MMA passes per 4096-point
     transform, fp16 operands, fp32 accumulation) meets the bf16 bar as well:
