@@ -34,7 +34,8 @@
 // power-of-two factors are gathered into the slice's P scale.
 //
 // All waits on the MMA mbarrier are bounded; a timeout sets bit 0 of the
-// device error word and the block stops after releasing its tensor memory.
+// device error word and the block stops after releasing its tensor memory
+// (results of that run are invalid).
 #include <cuda_fp16.h>
 
 #include "fft_regs.cuh"
@@ -81,10 +82,13 @@ __device__ __forceinline__ int scale_shift(float m) {
 
 struct Mma {
     uint32_t tile, op, mbar, dcol, phase;
-    int *flag;
+    bool late;   // this thread's last wait gave up
 
-    // One elected thread issues the chain and waits for its commit; every
-    // thread learns whether the wait completed.  full_n: all 128 result
+    // One elected thread issues the chain after a block barrier; every thread
+    // then waits for the commit's mbarrier phase itself (bounded), so no second
+    // barrier is needed.  A wait that gave up anywhere is seen by the whole
+    // block at the next issue barrier (run returns false, uniformly) or in
+    // any_late().  full_n: all 128 result
     // columns, over the K steps (16 reals each) whose bit is set in ksteps.
     // Otherwise all 8 K steps, and for each group g in gmask the 16 result
     // columns of DFT-matrix rows 16 g .. 16 g + 15 (outputs 8 g .. 8 g + 7),
@@ -92,7 +96,7 @@ struct Mma {
     __device__ __forceinline__ bool run(uint32_t ksteps, uint32_t gmask, bool full_n) {
         tc::fence_proxy_async();
         tc::fence_before();
-        __syncthreads();
+        if (__syncthreads_or(late)) return false;
         if (threadIdx.x == 0) {
             tc::fence_after();
             if (full_n) {
@@ -116,13 +120,15 @@ struct Mma {
                 }
             }
             tc::commit(mbar);
-            if (!tc::mbar_wait(mbar, phase, kWaitLimit)) *flag = 1;
         }
+        late = !tc::mbar_wait(mbar, phase, kWaitLimit);
         phase ^= 1u;
-        const bool ok = __syncthreads_and(*flag == 0);
         tc::fence_after();
-        return ok;
+        return true;
     }
+
+    // whether any thread's last wait gave up (a block-wide barrier)
+    __device__ __forceinline__ bool any_late() { return __syncthreads_or(late); }
 };
 
 // Pass-1 epilogue shared by all four transforms: read this thread's half row
@@ -176,7 +182,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
     uint64_t *mbar = reinterpret_cast<uint64_t *>(op + kOpBytes);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);   // [0] D, [1] S
     float *red = reinterpret_cast<float *>(tslot + 2);           // per-warp maxima
-    int *flag = reinterpret_cast<int *>(red + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
@@ -188,10 +193,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
         tc::tmem_alloc_keep(&tslot[1], kSCols);
         tc::tmem_relinquish();
     }
-    if (tid == 0) {
-        tc::mbar_init(tc::smem_u32(mbar), 1);
-        *flag = 0;
-    }
+    if (tid == 0) tc::mbar_init(tc::smem_u32(mbar), 1);
     {
         const uint4 *src = static_cast<const uint4 *>(a.w64op);
         uint4 *dst = reinterpret_cast<uint4 *>(op);
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
     mma.mbar = tc::smem_u32(mbar);
     mma.dcol = tslot[0];
     mma.phase = 0;
-    mma.flag = flag;
+    mma.late = false;
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
     const uint32_t tlD = tslot[0] + lane_base;
     const uint32_t tlS = tslot[1] + lane_base;
@@ -398,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
                 a.pscale[2 * pslice + (cc & 1)] = ldexpf(1.0f, min(127, 48 - shift_sum));
         }
     }
+    if (mma.any_late()) abort = true;   // also a timeout in the last wait
     if (abort && tid == 0 && a.err) atomicOr(a.err, 1);
     tc::fence_before();
     __syncthreads();
