@@ -50,14 +50,42 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed: what the
+    compiler sees, so editing a comment does not change the hash."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":                       # string or character literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash() -> str:
+    """Hash of the library's code (csrc/ and include/, comments and whitespace
+    ignored); the ncu traffic in profiles/traffic.txt is used only under the
+    hash it was captured on."""
     files = sorted(glob.glob(os.path.join(ROOT, "sub_quadratic_attention_b200", "csrc", "*")) +
                    glob.glob(os.path.join(ROOT, "include", "*.h")))
     h = hashlib.sha1()
     for f in files:
-        with open(f, "rb") as fh:
+        with open(f, encoding="utf-8", errors="replace") as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -1,14 +1,16 @@
-// kernels.cu -- the three kernel families of the SPECTRE spectral mixer on
+// kernels.cu -- the CUDA-core kernels of the SPECTRE spectral mixer on
 // sm_100a (SPECTRE walk-through, hotelren.com/news/5925787: §2.2 pseudocode,
 // §2.3 truncation, §3.1 real/imaginary parts carried as separate reals).
 //
-//   spectre_rows_fwd    : q, k, v rows -> R-point real transforms -> A
-//   spectre_slices<M>   : per (b, c, f1) slice: three M-point FFTs, the gated
-//                         product, one inverse M-point FFT -> P
-//   spectre_rows_inv_ln : P -> R-point inverse (real output) -> + x ->
-//                         LayerNorm over C -> y
+//   spectre_rows_fwd[_pipe]     : q, k, v rows -> R-point real transforms -> A
+//   spectre_slices<M>           : per (b, c, f1) slice: three M-point FFTs, the
+//                                 gated product, one inverse M-point FFT -> P
+//   spectre_rows_inv_ln[_reg|_pipe] : P -> R-point inverse (real output) -> + x
+//                                 -> LayerNorm over C -> y
 //
-// The index algebra is in kernels.cuh.
+// The _pipe variants are persistent and prefetch their next work item into
+// shared memory with cp.async.  The tensor-core slice pass for M = 4096 is in
+// slices_mma.cu.  The index algebra is in kernels.cuh.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 

@@ -1,5 +1,6 @@
-// kernels.cuh -- launch interface between the plan (api.cu) and the three
-// kernel families of the SPECTRE mixer (rows_fwd.cu, slices.cu, rows_inv_ln.cu).
+// kernels.cuh -- launch interface between the plan (api.cu) and the kernels
+// of the SPECTRE mixer (kernels.cu: row passes, CUDA-core slice pass, inverse
+// passes; slices_mma.cu: tensor-core slice pass).
 //
 // Decomposition (four-step Cooley-Tukey along L, split L = R * M, token
 // t = t1 * M + t2, rfft bin f = f1 + R * f2):
