@@ -51,7 +51,8 @@ def _load():
         lib.oracle_spectre_out.restype = ctypes.c_int
         lib.oracle_spectre_mix.argtypes = [
             ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_long, vp, vp, ctypes.c_int]
+            ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_long, vp, vp, ctypes.c_int,
+            ctypes.c_int]
         lib.oracle_spectre_mix.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -128,12 +129,18 @@ def spectre_out(q, k, v, G, H: int, F: int, c0: int = 0, c1: Optional[int] = Non
     return out
 
 
+NORM_MODES = {"post_ln": 0, "pre_ln": 1, "post_rms": 2, "pre_rms": 3}
+
+
 def spectre_mix(q, k, v, x, G, gamma, beta, H: int, F: int, eps: float = 1e-5,
-                tokens: Optional[Sequence[int]] = None, nthreads: int = 0):
+                tokens: Optional[Sequence[int]] = None, nthreads: int = 0, norm: str = "post_ln"):
     """Return ``(out, y)`` in float64 at the selected tokens (all if None).
 
     Shapes: ``out`` and ``y`` are ``[B, ntok, C]``.  ``eps`` is taken as the
-    fp32 value the library receives, widened to double.
+    fp32 value the library receives, widened to double.  ``norm``: "post_ln"
+    y = LN(out + x) (walk-through §2.2), "pre_ln" y = LN(out) + x, "post_rms"
+    y = RMS(out + x), "pre_rms" y = RMS(out) + x (the §3.3 variants), with
+    RMS(z) = z / sqrt(mean(z^2) + eps) * gamma + beta.
     """
     qa, dt = _as_stored(q)
     ka, _ = _as_stored(k)
@@ -158,7 +165,7 @@ def spectre_mix(q, k, v, x, G, gamma, beta, H: int, F: int, eps: float = 1e-5,
     rc = _load().oracle_spectre_mix(B, L, H, D, F, dt, eps64, _ptr(qa), _ptr(ka), _ptr(va),
                                     _ptr(xa), _ptr(Ga), _ptr(ga), _ptr(ba),
                                     None if tok is None else _ptr(tok), ntok,
-                                    _ptr(out), _ptr(y), nthreads)
+                                    _ptr(out), _ptr(y), nthreads, NORM_MODES[norm])
     if rc != 0:
         raise RuntimeError("oracle_spectre_mix failed")
     return out, y

@@ -297,23 +297,27 @@ int oracle_spectre_out(int B, long L, int H, int D, int F, int dtype,
 
 /*
  * oracle_spectre_mix: y = LayerNorm_C(out + x) at selected tokens
- * (SPECTRE walk-through §2.2: layer_norm(out + x)).
+ * (SPECTRE walk-through §2.2: layer_norm(out + x)), or one of the variants
+ * the walk-through's §3.3 names (normalise before the residual; RMSNorm).
  *   tok: ntok token indices in [0, L) (NULL with ntok = L means every token).
  *   out_sel: [B, ntok, C] double or NULL; y_sel: [B, ntok, C] double.
- * LayerNorm: mean and biased variance over the C channels of one token,
- * y = (z - mean) / sqrt(var + eps) * gamma + beta.
+ *   norm_mode: 0 y = LN(out + x); 1 y = LN(out) + x;
+ *              2 y = RMS(out + x); 3 y = RMS(out) + x.
+ * LN(z) = (z - mean) / sqrt(var + eps) * gamma + beta, mean and biased
+ * variance over the C channels of one token; RMS(z) = z / sqrt(mean(z^2) +
+ * eps) * gamma + beta.
  */
 int oracle_spectre_mix(int B, long L, int H, int D, int F, int dtype,
                        double eps, const void *q, const void *k,
                        const void *v, const void *x, const float *G,
                        const float *gamma, const float *beta,
                        const long *tok, long ntok, double *out_sel,
-                       double *y_sel, int nthreads)
+                       double *y_sel, int nthreads, int norm_mode)
 {
     long C = (long)H * D;
     long nb = L / 2 + 1;
     if (B < 1 || L < 2 || H < 1 || D < 1 || F < 1 || F > nb || ntok < 1 ||
-        (dtype != 0 && dtype != 1) || !y_sel)
+        (dtype != 0 && dtype != 1) || !y_sel || norm_mode < 0 || norm_mode > 3)
         return -1;
     if (!tok && ntok != L) return -1;
     for (long i = 0; tok && i < ntok; i++)
@@ -363,25 +367,32 @@ int oracle_spectre_mix(int B, long L, int H, int D, int F, int dtype,
         return -1;
     }
 
-    /* residual + LayerNorm over C, token by token */
+    /* residual and normalisation over C, token by token */
+    const int pre = norm_mode & 1, rms = norm_mode >> 1;
     for (long b = 0; b < B; b++) {
         for (long i = 0; i < ntok; i++) {
             long t = tok ? tok[i] : i;
             const double *orow = o + ((size_t)b * (size_t)ntok + (size_t)i) * (size_t)C;
             double *yrow = y_sel + ((size_t)b * (size_t)ntok + (size_t)i) * (size_t)C;
             size_t xbase = ((size_t)b * (size_t)L + (size_t)t) * (size_t)C;
-            double mean = 0.0;
-            for (long c = 0; c < C; c++) {
-                yrow[c] = orow[c] + load_elem(x, xbase + (size_t)c, dtype);
-                mean += yrow[c];
-            }
-            mean /= (double)C;
-            double var = 0.0;
-            for (long c = 0; c < C; c++) var += (yrow[c] - mean) * (yrow[c] - mean);
-            var /= (double)C;
-            double rstd = 1.0 / sqrt(var + eps);
+            /* z: out + x, or out alone when x is added after the norm */
             for (long c = 0; c < C; c++)
+                yrow[c] = orow[c] + (pre ? 0.0 : load_elem(x, xbase + (size_t)c, dtype));
+            double mean = 0.0, var = 0.0;
+            if (rms) {
+                for (long c = 0; c < C; c++) var += yrow[c] * yrow[c];
+                var /= (double)C;                       /* mean of squares */
+            } else {
+                for (long c = 0; c < C; c++) mean += yrow[c];
+                mean /= (double)C;
+                for (long c = 0; c < C; c++) var += (yrow[c] - mean) * (yrow[c] - mean);
+                var /= (double)C;
+            }
+            double rstd = 1.0 / sqrt(var + eps);
+            for (long c = 0; c < C; c++) {
                 yrow[c] = (yrow[c] - mean) * rstd * (double)gamma[c] + (double)beta[c];
+                if (pre) yrow[c] += load_elem(x, xbase + (size_t)c, dtype);
+            }
         }
     }
     if (!out_sel) free(o);

@@ -212,6 +212,54 @@ def test_shift_equivariance_and_trilinearity():
     assert np.max(np.abs(scaled - 2.0 * base)) < 1e-12 * np.max(np.abs(base))
 
 
+@pytest.mark.parametrize("norm", ["pre_ln", "post_rms", "pre_rms"])
+def test_norm_variants_match_torch_on_oracle_out(norm):
+    """The norm-order and RMSNorm variants (walk-through §3.3) against torch's
+    layer_norm / rms_norm applied to the oracle's own pre-norm output; out
+    itself does not depend on the variant."""
+    B, L, H, D = 2, 32, 2, 5
+    C = H * D
+    q, k, v, x = _mk(B, L, C, seed=13)
+    G = torch.rand(H, L // 2 + 1, generator=torch.Generator().manual_seed(7))
+    gamma = torch.randn(C, generator=torch.Generator().manual_seed(8))
+    beta = torch.randn(C, generator=torch.Generator().manual_seed(9))
+    out0, _ = oracle.spectre_mix(q, k, v, x, G, gamma, beta, H=H, F=11)
+    out, y = oracle.spectre_mix(q, k, v, x, G, gamma, beta, H=H, F=11, norm=norm)
+    assert np.array_equal(out, out0)
+    eps = float(np.float32(1e-5))
+    o = torch.from_numpy(out)
+    xd, g, bt = x.double(), gamma.double(), beta.double()
+    F_ = torch.nn.functional
+    if norm == "pre_ln":
+        ref = F_.layer_norm(o, (C,), g, bt, eps=eps) + xd
+    elif norm == "post_rms":
+        ref = F_.rms_norm(o + xd, (C,), g, eps=eps) + bt
+    else:
+        ref = F_.rms_norm(o, (C,), g, eps=eps) + bt + xd
+    assert np.max(np.abs(y - ref.numpy())) < 1e-12
+
+
+def test_rmsnorm_equals_layernorm_on_zero_mean_tokens():
+    """With x chosen so that every token's z = out + x has zero channel mean,
+    RMS(z) and LN(z) coincide: pins the one step in which they differ."""
+    B, L, H, D = 1, 64, 2, 4
+    C = H * D
+    q, k, v, x = _mk(B, L, C, seed=21)
+    q, k, v, x = q.double(), k.double(), v.double(), x.double()
+    G = torch.rand(H, L // 2 + 1, generator=torch.Generator().manual_seed(3), dtype=torch.float64)
+    gamma = torch.randn(C, generator=torch.Generator().manual_seed(4))
+    beta = torch.randn(C, generator=torch.Generator().manual_seed(5))
+    out, _ = oracle.spectre_mix(q.float(), k.float(), v.float(), x.float(), G.float(), gamma, beta,
+                                H=H, F=L // 2 + 1)
+    z = torch.from_numpy(out) + x
+    x0 = (x - z.mean(dim=-1, keepdim=True)).float()     # z + (x0 - x) has mean ~ 0
+    _, y_ln = oracle.spectre_mix(q.float(), k.float(), v.float(), x0, G.float(), gamma, beta,
+                                 H=H, F=L // 2 + 1, norm="post_ln")
+    _, y_rms = oracle.spectre_mix(q.float(), k.float(), v.float(), x0, G.float(), gamma, beta,
+                                  H=H, F=L // 2 + 1, norm="post_rms")
+    assert np.max(np.abs(y_ln - y_rms)) < 1e-5
+
+
 def test_layernorm_matches_torch_on_oracle_z():
     B, L, H, D = 2, 32, 2, 5
     C = H * D
