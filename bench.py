@@ -271,7 +271,8 @@ def native_arm(args, w, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps,
-                             tensor_cores=False if args.cuda_core_slices else None)
+                             tensor_cores=False if args.cuda_core_slices else None,
+                             norm=args.norm)
     h = mix.handle
 
     def barrier():
@@ -384,7 +385,7 @@ def native_arm(args, w, rank, world, local_rank):
                         "row pass with the previous chunk's slice pass on two streams",
         "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
                  "chunks": nchunks, "launches_per_step": nlaunch,
-                 "slice_pass": mix.slice_pass},
+                 "slice_pass": mix.slice_pass, "norm": args.norm},
     }
 
     # ---- CPU baseline (rank 0, N = 1 only)
@@ -432,6 +433,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--norm", choices=["post_ln", "pre_ln", "post_rms", "pre_rms"], default="post_ln",
+                    help="normalisation: LayerNorm(out + x) (default), LayerNorm(out) + x, or the "
+                         "RMSNorm forms")
     ap.add_argument("--cuda-core-slices", action="store_true",
                     help="force the CUDA-core slice pass (plan option; default: tensor cores "
                          "where the plan allows)")

@@ -180,7 +180,22 @@ enum spectre_option {
      * the truncation pruning the MMAs.  0: the CUDA-core slice pass (fp32
      * Stockham radix-16 butterflies) for every plan.  Plans outside the
      * tensor-core range always take the CUDA-core pass. */
-    SPECTRE_OPT_TENSOR_CORES = 1
+    SPECTRE_OPT_TENSOR_CORES = 1,
+    /* How the mixer output is normalised (enum spectre_norm; default
+     * SPECTRE_NORM_POST_LN, the walk-through's §2.2 form).  The other values
+     * are the §3.3 variants.  The no-allocation entry point always uses the
+     * default. */
+    SPECTRE_OPT_NORM = 2
+};
+
+enum spectre_norm {
+    SPECTRE_NORM_POST_LN = 0,   /* y = LayerNorm(out + x) */
+    SPECTRE_NORM_PRE_LN = 1,    /* y = LayerNorm(out) + x */
+    SPECTRE_NORM_POST_RMS = 2,  /* y = RMSNorm(out + x) */
+    SPECTRE_NORM_PRE_RMS = 3    /* y = RMSNorm(out) + x */
+    /* LayerNorm(z) = (z - mean) / sqrt(var + eps) * gamma + beta (biased
+     * variance over C); RMSNorm(z) = z / sqrt(mean(z^2) + eps) * gamma + beta
+     * (pass beta = 0 for the usual bias-free form). */
 };
 
 /* Set an option of the plan (see enum spectre_option).  Takes effect for

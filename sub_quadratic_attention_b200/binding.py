@@ -27,6 +27,10 @@ SPECTRE_ERR_SCRATCH = -7
 SPECTRE_ERR_TIMEOUT = -8
 
 SPECTRE_OPT_TENSOR_CORES = 1
+SPECTRE_OPT_NORM = 2
+
+# enum spectre_norm, keyed as in the oracle
+SPECTRE_NORM = {"post_ln": 0, "pre_ln": 1, "post_rms": 2, "pre_rms": 3}
 
 SPECTRE_SLICE_CUDA_CORES = 0
 SPECTRE_SLICE_TENSOR_CORES = 1
@@ -206,7 +210,8 @@ class SpectreMix:
     """
 
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
-                 dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None):
+                 dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None,
+                 norm: Optional[str] = None):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
         self.F = L // 2 + 1 if F is None else F
@@ -215,6 +220,8 @@ class SpectreMix:
         self.handle = spectre_mix_create(B, L, H, D, self.F, self.dtype_code, eps)
         if tensor_cores is not None:   # None keeps the library's default (on)
             spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1 if tensor_cores else 0)
+        if norm is not None:           # None keeps the default, "post_ln": LayerNorm(out + x)
+            spectre_mix_set_option(self.handle, SPECTRE_OPT_NORM, SPECTRE_NORM[norm])
 
     def __call__(self, q, k, v, x, G, gamma, beta, y=None, out=None, stream=None):
         import torch

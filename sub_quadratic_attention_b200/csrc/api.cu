@@ -26,6 +26,7 @@ struct PathGeom {
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
     int tc_mode;         // option: slice pass on the tensor cores where mma_ok (1) or CUDA cores (0)
+    int norm_mode;       // option: enum spectre_norm
     int mma_ok;          // the DFT-64 MMA slice pass applies (M = 4096, fp16 P, few live groups)
     int nsm;             // multiprocessors of the device
     int chunk;           // channels per pipeline chunk (multiple of 64, or C)
@@ -194,6 +195,7 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
         g->mma_ok = worst <= kMmaMaxGroups ? 1 : 0;
     }
     g->tc_mode = 1;
+    g->norm_mode = SPECTRE_NORM_POST_LN;
     g->nsm = 148;
     // pipeline chunks: four channel chunks when each still fills the GPU
     g->chunk = C;
@@ -295,6 +297,7 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     ia.reg_variant = g.inv_reg;
     ia.vec2 = (g.C % 2 == 0) ? 1 : 0;
     ia.nsm = g.nsm;
+    ia.norm = g.norm_mode;
     e = mark(s);
     if (e == cudaSuccess) e = launch_rows_inv_ln(g.R, g.dtype, ia, s);
     if (e == cudaSuccess) e = mark(s);
@@ -654,6 +657,10 @@ int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     case SPECTRE_OPT_TENSOR_CORES:
         if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
         h->g.tc_mode = value;
+        return SPECTRE_OK;
+    case SPECTRE_OPT_NORM:
+        if (value < SPECTRE_NORM_POST_LN || value > SPECTRE_NORM_PRE_RMS) return SPECTRE_ERR_ARG;
+        h->g.norm_mode = value;
         return SPECTRE_OK;
     default: return SPECTRE_ERR_ARG;
     }

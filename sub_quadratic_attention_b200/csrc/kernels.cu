@@ -536,7 +536,9 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
 // ---------------------------------------------------------------------------
 // inverse row pass + residual + LayerNorm
 // ---------------------------------------------------------------------------
-template <int R, typename T, bool DEBUG_OUT>
+// NV: the plan uses a norm variant (residual after the norm, or RMSNorm);
+// without it the default LayerNorm(out + x) code is compiled alone.
+template <int R, typename T, bool DEBUG_OUT, bool NV>
 __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
     constexpr bool P16 = std::is_same<T, __nv_bfloat16>::value;  // bf16 I/O: fp16 P
@@ -604,6 +606,7 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
     const T *x = static_cast<const T *>(a.x);
     T *y = static_cast<T *>(a.y);
     const float invC = 1.0f / (float)a.C;
+    const bool pre = NV && (a.norm & 1), rms = NV && ((a.norm >> 1) & 1);   // residual after the norm; RMSNorm
     for (int row = warp; row < R * T2C; row += nw) {
         const int t1 = row / T2C, tl = row % T2C;
         const int t2 = t2base + tl;
@@ -616,19 +619,27 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
         for (int c = lane; c < a.C; c += 32) {
             float o = zr[c];
             if (DEBUG_OUT) a.out_f32[tok * a.C + c] = o;
-            float z = o + Elem<T>::load(xr + c);
+            float z = pre ? o : o + Elem<T>::load(xr + c);
             zr[c] = z;
-            s += z;
+            s = rms ? fmaf(z, z, s) : s + z;
         }
-        const float mean = warp_sum(s) * invC;
-        float ss = 0.f;
+        float mean = 0.f, rstd;
+        if (rms) {
+            rstd = rsqrtf(warp_sum(s) * invC + a.eps);
+        } else {
+            mean = warp_sum(s) * invC;
+            float ss = 0.f;
+            for (int c = lane; c < a.C; c += 32) {
+                float d = zr[c] - mean;
+                ss = fmaf(d, d, ss);
+            }
+            rstd = rsqrtf(warp_sum(ss) * invC + a.eps);
+        }
         for (int c = lane; c < a.C; c += 32) {
-            float d = zr[c] - mean;
-            ss = fmaf(d, d, ss);
+            float yv = fmaf((zr[c] - mean) * rstd, __ldg(a.gamma + c), __ldg(a.beta + c));
+            if (pre) yv += Elem<T>::load(xr + c);
+            Elem<T>::store(yr + c, yv);
         }
-        const float rstd = rsqrtf(warp_sum(ss) * invC + a.eps);
-        for (int c = lane; c < a.C; c += 32)
-            Elem<T>::store(yr + c, fmaf((zr[c] - mean) * rstd, __ldg(a.gamma + c), __ldg(a.beta + c)));
     }
 }
 
@@ -668,7 +679,7 @@ template <int N, int BIT, int BITEND> struct HalvingReduce {
 
 constexpr int ilog2c(int v) { return v <= 1 ? 0 : 1 + ilog2c(v / 2); }
 
-template <int R, int T2C, typename T, bool DEBUG_OUT>
+template <int R, int T2C, typename T, bool DEBUG_OUT, bool NV>
 __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
     constexpr bool P16 = std::is_same<T, __nv_bfloat16>::value;  // bf16 I/O: fp16 P
@@ -734,6 +745,7 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     const size_t tok0 = (size_t)b * a.L + (live ? t2 : 0);
     const int rowstep = a.M * a.C;                      // elements between t1 rows
     const T *xp = x + tok0 * a.C + (live ? c0 : 0);
+    const bool pre = NV && (a.norm & 1), rms = NV && ((a.norm >> 1) & 1);   // residual after the norm; RMSNorm
     float s[R];
 #pragma unroll
     for (int t1 = 0; t1 < R; t1++) {
@@ -746,7 +758,10 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
                 if (has1) op[1] = z1[t1];
             }
         }
-        if (has1 && a.vec2) {
+        if (pre) {
+            z0[t1] = live ? z0[t1] : 0.f;
+            z1[t1] = has1 ? z1[t1] : 0.f;
+        } else if (has1 && a.vec2) {
             float2 xv = Elem<T>::load2(xp + t1 * rowstep);
             z0[t1] += xv.x;
             z1[t1] += xv.y;
@@ -754,13 +769,15 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
             z0[t1] = live ? z0[t1] + Elem<T>::load(xp + t1 * rowstep) : 0.f;
             z1[t1] = has1 ? z1[t1] + Elem<T>::load(xp + t1 * rowstep + 1) : 0.f;
         }
-        s[t1] = z0[t1] + z1[t1];
+        s[t1] = rms ? fmaf(z0[t1], z0[t1], z1[t1] * z1[t1]) : z0[t1] + z1[t1];
     }
     const float invC = 1.0f / (float)a.C;
-    // two reductions over the channels of each row: sum(z), then sum((z - mean)^2);
-    // stat[0][.] holds the means, stat[1][.] the reciprocal standard deviations
+    // two reductions over the channels of each row: sum(z), then sum((z - mean)^2)
+    // (RMSNorm: one, sum(z^2)); stat[0][.] holds the means (0 for RMSNorm),
+    // stat[1][.] the reciprocal standard deviations
+    const int npass = rms ? 1 : 2;
 #pragma unroll 1
-    for (int pass = 0; pass < 2; pass++) {
+    for (int pass = 0; pass < npass; pass++) {
         if (pass == 1) {
 #pragma unroll
             for (int t1 = 0; t1 < R; t1++) {
@@ -787,7 +804,14 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
         for (int i = warp; i < T2C * R; i += nwarps) {
             float acc = lane < nwarps ? part[i * PS + lane] : 0.f;
             acc = warp_sum(acc) * invC;
-            if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
+            if (lane == 0) {
+                if (rms) {
+                    stat[i] = 0.f;
+                    stat[T2C * R + i] = rsqrtf(acc + a.eps);
+                } else {
+                    stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
+                }
+            }
         }
         __syncthreads();
     }
@@ -799,8 +823,18 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
     for (int t1 = 0; t1 < R; t1++) {
         const float mu = stat[tl * R + t1];
         const float rstd = stat[T2C * R + tl * R + t1];
-        const float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
-        const float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
+        float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
+        float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
+        if (pre) {
+            if (has1 && a.vec2) {
+                const float2 xv = Elem<T>::load2(xp + t1 * rowstep);
+                y0 += xv.x;
+                y1 += xv.y;
+            } else {
+                if (live) y0 += Elem<T>::load(xp + t1 * rowstep);
+                if (has1) y1 += Elem<T>::load(xp + t1 * rowstep + 1);
+            }
+        }
         if (has1 && a.vec2) {
             Elem<T>::store2(yp + t1 * rowstep, y0, y1);
         } else if (live) {
@@ -830,7 +864,7 @@ __host__ __device__ inline int inv_pipe_stage_words(int C) {
     return 9 * (C / 2) * 2 * 2 + 16 * 2 * (C + 32) / 2;
 }
 
-template <bool DEBUG_OUT>
+template <bool DEBUG_OUT, bool NV>
 __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(RowsInvArgs a) {
     constexpr int R = 16, NF = R / 2 + 1, T2C = 2;
     extern __shared__ float4 smem_f4[];
@@ -875,6 +909,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     const float g0 = live ? __ldg(a.gamma + c0) : 0.f, be0 = live ? __ldg(a.beta + c0) : 0.f;
     const float g1 = live ? __ldg(a.gamma + c0 + 1) : 0.f, be1 = live ? __ldg(a.beta + c0 + 1) : 0.f;
     const float invC = 1.0f / (float)C;
+    const bool pre = NV && (a.norm & 1), rms = NV && ((a.norm >> 1) & 1);   // residual after the norm; RMSNorm
     long long grp = blockIdx.x;
     if (grp < ngroups) prefetch(grp, 0);
     cp_async_commit();
@@ -921,16 +956,17 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
                 if (DEBUG_OUT && live)
                     *reinterpret_cast<float2 *>(a.out_f32 + (tok0 + (size_t)t1 * a.M) * C + c0) =
                         make_float2(z0[t1], z1[t1]);
-                const uint32_t xw = live ? xst[(t1 * 2 + tl) * (XS / 2) + cp] : 0u;
+                const uint32_t xw = (live && !pre) ? xst[(t1 * 2 + tl) * (XS / 2) + cp] : 0u;
                 const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw));
                 z0[t1] = live ? z0[t1] + xv.x : 0.f;
                 z1[t1] = live ? z1[t1] + xv.y : 0.f;
-                s[t1] = z0[t1] + z1[t1];
+                s[t1] = rms ? fmaf(z0[t1], z0[t1], z1[t1] * z1[t1]) : z0[t1] + z1[t1];
             }
         }
-        // LayerNorm statistics of the 2 x R token rows, two passes
+        // statistics of the 2 x R token rows: mean, then mean squared
+        // deviation (RMSNorm: the mean square alone)
 #pragma unroll 1
-        for (int pass = 0; pass < 2; pass++) {
+        for (int pass = 0; pass < (rms ? 1 : 2); pass++) {
             if (pass == 1) {
 #pragma unroll
                 for (int t1 = 0; t1 < R; t1++) {
@@ -952,7 +988,14 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
             for (int i = warp; i < T2C * R; i += nwarps) {
                 float acc = lane < nwarps ? part[i * PS + lane] : 0.f;
                 acc = warp_sum(acc) * invC;
-                if (lane == 0) stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
+                if (lane == 0) {
+                    if (rms) {
+                        stat[i] = 0.f;
+                        stat[T2C * R + i] = rsqrtf(acc + a.eps);
+                    } else {
+                        stat[pass * T2C * R + i] = pass == 0 ? acc : rsqrtf(acc + a.eps);
+                    }
+                }
             }
             __syncthreads();
         }
@@ -961,8 +1004,15 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
 #pragma unroll
             for (int t1 = 0; t1 < R; t1++) {
                 const float mu = stat[tl * R + t1], rstd = stat[T2C * R + tl * R + t1];
-                Elem<__nv_bfloat16>::store2(yp + t1 * rowstep, fmaf((z0[t1] - mu) * rstd, g0, be0),
-                                            fmaf((z1[t1] - mu) * rstd, g1, be1));
+                float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
+                float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
+                if (pre) {   // the residual, still in this stage
+                    const uint32_t xw = xst[(t1 * 2 + tl) * (XS / 2) + cp];
+                    const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw));
+                    y0 += xv.x;
+                    y1 += xv.y;
+                }
+                Elem<__nv_bfloat16>::store2(yp + t1 * rowstep, y0, y1);
             }
         }
         // every read of this stage and of stat is done before the stage is refilled
@@ -1060,13 +1110,22 @@ void slice_geometry(int M, int *nt, int *spb, size_t *smem) {
     }
 }
 
+template <int R, typename T, bool NV>
+static cudaError_t rows_inv_RTV(const RowsInvArgs &a, cudaStream_t s);
+
+// NV selects the build of each inverse kernel that handles the norm variants
 template <int R, typename T>
 static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
+    return a.norm != 0 ? rows_inv_RTV<R, T, true>(a, s) : rows_inv_RTV<R, T, false>(a, s);
+}
+
+template <int R, typename T, bool NV>
+static cudaError_t rows_inv_RTV(const RowsInvArgs &a, cudaStream_t s) {
     if constexpr (R == 16 && std::is_same<T, __nv_bfloat16>::value) {
         if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0) {
             const int threads = ((a.C + 31) / 32) * 32;         // 2 columns x C / 2 pairs
             const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32 + 1) * 32 + 64) * 4;
-            auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true> : spectre_rows_inv_ln_pipe<false>;
+            auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true, NV> : spectre_rows_inv_ln_pipe<false, NV>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             int per_sm = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess ||
@@ -1084,12 +1143,12 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
         const int threads = ((a.T2C * CP + 31) / 32) * 32;
         size_t smem = (size_t)((threads / 32 + 1) * a.T2C * R + 2 * a.T2C * R) * sizeof(float);
         switch (a.T2C) {
-#define SPECTRE_INV_T2C(t2c)                                                          \
-    case t2c:                                                                         \
-        if (a.out_f32)                                                                \
-            spectre_rows_inv_ln_reg<R, t2c, T, true><<<grid, threads, smem, s>>>(a);  \
-        else                                                                          \
-            spectre_rows_inv_ln_reg<R, t2c, T, false><<<grid, threads, smem, s>>>(a); \
+#define SPECTRE_INV_T2C(t2c)                                                              \
+    case t2c:                                                                             \
+        if (a.out_f32)                                                                    \
+            spectre_rows_inv_ln_reg<R, t2c, T, true, NV><<<grid, threads, smem, s>>>(a);  \
+        else                                                                              \
+            spectre_rows_inv_ln_reg<R, t2c, T, false, NV><<<grid, threads, smem, s>>>(a); \
         break;
             SPECTRE_INV_T2C(1) SPECTRE_INV_T2C(2) SPECTRE_INV_T2C(4) SPECTRE_INV_T2C(8)
 #undef SPECTRE_INV_T2C
@@ -1100,11 +1159,11 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
     dim3 grid((a.M + a.T2C - 1) / a.T2C, a.B);
     size_t smem = (size_t)R * a.T2C * a.ZS * sizeof(float);
     if (a.out_f32) {
-        auto k = spectre_rows_inv_ln<R, T, true>;
+        auto k = spectre_rows_inv_ln<R, T, true, NV>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, 512, smem, s>>>(a);
     } else {
-        auto k = spectre_rows_inv_ln<R, T, false>;
+        auto k = spectre_rows_inv_ln<R, T, false, NV>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, 512, smem, s>>>(a);
     }

@@ -82,6 +82,7 @@ struct RowsInvArgs {
     int reg_variant;      // 1: register-resident LayerNorm (R <= 16, C <= 2048)
     int vec2;             // C even: channel pairs as one vector
     int nsm;              // multiprocessors (grid of the persistent variant)
+    int norm;             // bit 0: residual after the norm; bit 1: RMSNorm (no mean)
     float eps;
 };
 

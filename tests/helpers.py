@@ -18,14 +18,15 @@ def to_device(inputs):
     return {k: v.cuda() for k, v in inputs.items()}
 
 
-def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None):
+def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None, norm=None):
     """Run the CUDA path through the C ABI.  Returns (out_f32 or None, y) on CPU.
     tensor_cores: None keeps the plan's default slice pass, True/False sets it."""
     from sub_quadratic_attention_b200 import binding
     from sub_quadratic_attention_b200.binding import SpectreMix
 
     d = to_device(inputs_cpu)
-    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps, tensor_cores=tensor_cores) as mix:
+    with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps, tensor_cores=tensor_cores,
+                    norm=norm) as mix:
         y = torch.empty_like(d["x"])
         out = torch.empty((w.B, w.L, w.C), dtype=torch.float32, device="cuda") if debug else None
         mix(d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y=y, out=out,
@@ -35,12 +36,12 @@ def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None):
     return (out.cpu() if debug else None), y.cpu()
 
 
-def oracle_full(w, inputs_cpu):
+def oracle_full(w, inputs_cpu, norm="post_ln"):
     import oracle
 
     return oracle.spectre_mix(inputs_cpu["q"], inputs_cpu["k"], inputs_cpu["v"], inputs_cpu["x"],
                               inputs_cpu["G"], inputs_cpu["gamma"], inputs_cpu["beta"],
-                              H=w.H, F=w.F, eps=w.eps)
+                              H=w.H, F=w.F, eps=w.eps, norm=norm)
 
 
 def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:

@@ -87,6 +87,7 @@ def test_null_handle_paths():
 
     assert b._lib.spectre_mix_set_option(None, b.SPECTRE_OPT_TENSOR_CORES, 1) == b.SPECTRE_ERR_ARG
     assert b._lib.spectre_mix_slice_pass(None) == b.SPECTRE_ERR_ARG
+    assert b._lib.spectre_mix_set_option(None, b.SPECTRE_OPT_NORM, 1) == b.SPECTRE_ERR_ARG
     assert b._lib.spectre_mix_device_status(None, None) == b.SPECTRE_ERR_ARG
     b.spectre_mix_destroy(None)                      # NULL-safe
     assert b.spectre_mix_workspace_bytes(None) == 0

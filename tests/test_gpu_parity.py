@@ -164,3 +164,22 @@ def test_run_rejects_misaligned_and_null_pointers():
         torch.cuda.synchronize()
     finally:
         b.spectre_mix_destroy(h)
+
+
+@pytest.mark.parametrize("norm", ["pre_ln", "post_rms", "pre_rms"])
+@pytest.mark.parametrize("case", ["bf16_long", "fp32_mid", (2, 4096, 3, 5, 700),
+                                  (1, 524288, 1, 4, 5000)])
+def test_norm_variants(norm, case):
+    """The norm-order and RMSNorm variants (walk-through §3.3) in every inverse
+    kernel: the prefetching one (bf16_long, with the tensor-core slice pass),
+    the register-resident one (fp32_mid; an odd channel count in bf16) and
+    the shared-memory one (R = 64, fp32)."""
+    if isinstance(case, str):
+        w = WORKLOADS[case]
+    else:
+        w = custom(*case, dtype="bf16" if case[1] == 4096 else "f32")
+    inp = make_inputs(w)
+    out, y = run_library(w, inp, norm=norm)
+    out_ref, y_ref = oracle_full(w, inp, norm=norm)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"{norm} {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
