@@ -47,12 +47,12 @@ def _load():
         lib.oracle_fft.restype = ctypes.c_int
         lib.oracle_spectre_out.argtypes = [
             ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-            vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int]
+            vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int]
         lib.oracle_spectre_out.restype = ctypes.c_int
         lib.oracle_spectre_mix.argtypes = [
             ctypes.c_int, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_long, vp, vp, ctypes.c_int,
-            ctypes.c_int]
+            ctypes.c_int, ctypes.c_int]
         lib.oracle_spectre_mix.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -81,6 +81,19 @@ def _as_stored(t):
     if a.dtype == np.float32:
         return a, 0
     raise TypeError(f"unsupported dtype {a.dtype}")
+
+
+def _gate(G):
+    """(float32 array, cgate): a real gate [H, L/2+1], or a complex one as
+    [H, L/2+1, 2] (re, im) pairs with cgate = 1."""
+    import torch
+
+    if isinstance(G, torch.Tensor) and G.is_complex():
+        return np.ascontiguousarray(torch.view_as_real(G.to(torch.complex64)).numpy()), 1
+    if isinstance(G, np.ndarray) and np.iscomplexobj(G):
+        a = np.stack([G.real, G.imag], axis=-1).astype(np.float32)
+        return np.ascontiguousarray(a), 1
+    return _f32(G), 0
 
 
 def _f32(t) -> np.ndarray:
@@ -120,10 +133,10 @@ def spectre_out(q, k, v, G, H: int, F: int, c0: int = 0, c1: Optional[int] = Non
         raise ValueError("C must be a multiple of H")
     D = C // H
     c1 = C if c1 is None else c1
-    Ga = _f32(G)
+    Ga, cg = _gate(G)
     out = np.empty((B, L, c1 - c0), dtype=np.float64)
     rc = _load().oracle_spectre_out(B, L, H, D, F, dt, _ptr(qa), _ptr(ka), _ptr(va), _ptr(Ga),
-                                    c0, c1, _ptr(out), nthreads)
+                                    c0, c1, _ptr(out), nthreads, cg)
     if rc != 0:
         raise RuntimeError("oracle_spectre_out failed")
     return out
@@ -150,7 +163,7 @@ def spectre_mix(q, k, v, x, G, gamma, beta, H: int, F: int, eps: float = 1e-5,
         raise TypeError("x must share q's dtype")
     B, L, C = qa.shape
     D = C // H
-    Ga = _f32(G)
+    Ga, cg = _gate(G)
     ga = _f32(gamma)
     ba = _f32(beta)
     if tokens is None:
@@ -165,7 +178,7 @@ def spectre_mix(q, k, v, x, G, gamma, beta, H: int, F: int, eps: float = 1e-5,
     rc = _load().oracle_spectre_mix(B, L, H, D, F, dt, eps64, _ptr(qa), _ptr(ka), _ptr(va),
                                     _ptr(xa), _ptr(Ga), _ptr(ga), _ptr(ba),
                                     None if tok is None else _ptr(tok), ntok,
-                                    _ptr(out), _ptr(y), nthreads, NORM_MODES[norm])
+                                    _ptr(out), _ptr(y), nthreads, NORM_MODES[norm], cg)
     if rc != 0:
         raise RuntimeError("oracle_spectre_mix failed")
     return out, y

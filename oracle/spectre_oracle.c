@@ -222,7 +222,7 @@ static void chan_ws_free(chan_ws *w)
 
 static void mix_channel(chan_ws *w, long b, long c, long L, long C, int D,
                         int F, int dtype, const void *q, const void *k,
-                        const void *v, const float *G)
+                        const void *v, const float *G, int cgate)
 {
     long nb = L / 2 + 1;
     size_t base = (size_t)b * (size_t)L * (size_t)C + (size_t)c;
@@ -232,12 +232,18 @@ static void mix_channel(chan_ws *w, long b, long c, long L, long C, int D,
     rfft(&w->ctx, w->col, w->K);
     for (long t = 0; t < L; t++) w->col[t] = load_elem(v, base + (size_t)t * C, dtype);
     rfft(&w->ctx, w->col, w->V);
-    const float *Gh = G + (size_t)(c / D) * (size_t)nb;
+    /* real gate: G[h][f]; complex gate (a relative-position phase, §2.4):
+     * G[h][f] = re + i im stored as pairs.  Bins f <= L/2 only: irfft
+     * extends O Hermitian-symmetrically, so the complex gate acts as
+     * conj(G[L - f]) above L/2 and the output stays real. */
+    const float *Gh = G + (size_t)(c / D) * (size_t)nb * (cgate ? 2 : 1);
     for (long f = 0; f < nb; f++) {
-        if (f < F)
-            w->Q[f] = w->Q[f] * conj(w->K[f]) * (double)Gh[f] * w->V[f];
-        else
+        if (f < F) {
+            cplx g = cgate ? (double)Gh[2 * f] + I * (double)Gh[2 * f + 1] : (double)Gh[f];
+            w->Q[f] = w->Q[f] * conj(w->K[f]) * g * w->V[f];
+        } else {
             w->Q[f] = 0.0;
+        }
     }
     irfft(&w->ctx, w->Q, w->oc);
 }
@@ -245,14 +251,15 @@ static void mix_channel(chan_ws *w, long b, long c, long L, long C, int D,
 /*
  * oracle_spectre_out: the pre-LayerNorm mixer output for a channel range.
  *   q, k, v: [B, L, C] in dtype (0 = fp32, 1 = bf16 bits), row-major.
- *   G: [H, L/2+1] fp32; channel c uses row c / D.
+ *   G: [H, L/2+1] fp32, or with cgate [H, L/2+1, 2] (re, im); channel c
+ *   uses row c / D.
  *   out: [B, L, c1 - c0] double (channel c written at column c - c0).
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
 int oracle_spectre_out(int B, long L, int H, int D, int F, int dtype,
                        const void *q, const void *k, const void *v,
                        const float *G, int c0, int c1, double *out,
-                       int nthreads)
+                       int nthreads, int cgate)
 {
     long C = (long)H * D;
     long nb = L / 2 + 1;
@@ -285,7 +292,7 @@ int oracle_spectre_out(int B, long L, int H, int D, int F, int dtype,
         for (long job = 0; job < njobs; job++) {
             if (!w.ok) continue;
             long b = job / W, c = c0 + job % W;
-            mix_channel(&w, b, c, L, C, D, F, dtype, q, k, v, G);
+            mix_channel(&w, b, c, L, C, D, F, dtype, q, k, v, G, cgate);
             for (long t = 0; t < L; t++)
                 out[((size_t)b * (size_t)L + (size_t)t) * (size_t)W + (size_t)(c - c0)] = w.oc[t];
         }
@@ -312,7 +319,7 @@ int oracle_spectre_mix(int B, long L, int H, int D, int F, int dtype,
                        const void *v, const void *x, const float *G,
                        const float *gamma, const float *beta,
                        const long *tok, long ntok, double *out_sel,
-                       double *y_sel, int nthreads, int norm_mode)
+                       double *y_sel, int nthreads, int norm_mode, int cgate)
 {
     long C = (long)H * D;
     long nb = L / 2 + 1;
@@ -353,7 +360,7 @@ int oracle_spectre_mix(int B, long L, int H, int D, int F, int dtype,
         for (long job = 0; job < njobs; job++) {
             if (!w.ok) continue;
             long b = job / C, c = job % C;
-            mix_channel(&w, b, c, L, C, D, F, dtype, q, k, v, G);
+            mix_channel(&w, b, c, L, C, D, F, dtype, q, k, v, G, cgate);
             for (long i = 0; i < ntok; i++) {
                 long t = tok ? tok[i] : i;
                 o[((size_t)b * (size_t)ntok + (size_t)i) * (size_t)C + (size_t)c] = w.oc[t];

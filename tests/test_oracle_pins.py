@@ -133,6 +133,67 @@ def test_mixer_matches_time_domain_general_gate(L, F):
         assert err < 1e-11, (c, err)
 
 
+def _complex_gate_kernel(Grow, F, L):
+    """g'[n] = (1/L) sum_f G'_f e^{2 pi i f n / L} for a complex gate given on
+    f <= L/2 (truncated at F), extended Hermitian-symmetrically
+    (G'_{L-f} = conj G'_f) with the imaginary parts at DC and Nyquist
+    dropped: a direct sum of cosines and sines."""
+    n = np.arange(L)
+    g = np.zeros(L)
+    for f in range(L // 2 + 1):
+        if f >= F:
+            continue
+        edge = f == 0 or (L % 2 == 0 and f == L // 2)
+        ph = 2 * np.pi * f * n / L
+        if edge:
+            g += Grow[f].real * np.cos(ph)
+        else:
+            g += 2.0 * (Grow[f].real * np.cos(ph) - Grow[f].imag * np.sin(ph))
+    return g / L
+
+
+@pytest.mark.parametrize("L,F", [(16, 9), (48, 11), (64, 33), (96, 20)])
+def test_complex_gate_matches_time_domain(L, F):
+    """A complex (phase-carrying) gate against the O(L^2) time-domain form."""
+    B, H, D = 1, 2, 2
+    C = H * D
+    q, k, v, _ = _mk(B, L, C, seed=2000 + L + F)
+    g = torch.Generator().manual_seed(L + F)
+    G = torch.complex(torch.rand(H, L // 2 + 1, generator=g), torch.randn(H, L // 2 + 1, generator=g))
+    out = oracle.spectre_out(q, k, v, G, H=H, F=F)
+    for c in range(C):
+        gk = _complex_gate_kernel(G[c // D].to(torch.complex128).numpy(), F, L)
+        ref = _time_domain_out(q[0, :, c].double().numpy(), k[0, :, c].double().numpy(),
+                               v[0, :, c].double().numpy(), gk)
+        err = np.max(np.abs(out[0, :, c] - ref)) / max(np.max(np.abs(ref)), 1e-300)
+        assert err < 1e-11, (c, err)
+
+
+def test_complex_gate_with_zero_phase_equals_real_gate():
+    B, L, H, D = 2, 64, 2, 3
+    C = H * D
+    q, k, v, _ = _mk(B, L, C, seed=31)
+    G = torch.rand(H, L // 2 + 1, generator=torch.Generator().manual_seed(2))
+    out_r = oracle.spectre_out(q, k, v, G, H=H, F=20)
+    out_c = oracle.spectre_out(q, k, v, torch.complex(G, torch.zeros_like(G)), H=H, F=20)
+    assert np.array_equal(out_r, out_c)
+
+
+@pytest.mark.parametrize("s", [1, 5, 17])
+def test_complex_gate_pure_delay_shifts_the_output(s):
+    """G_f = e^{-2 pi i f s / L}, no truncation: the gate kernel is a delta at
+    s, so the output is the identity-gate output delayed by s tokens."""
+    B, L, H, D = 1, 64, 1, 3
+    C = H * D
+    q, k, v, _ = _mk(B, L, C, seed=40 + s)
+    f = np.arange(L // 2 + 1)
+    ph = torch.from_numpy(np.exp(-2j * np.pi * f * s / L)).to(torch.complex64)[None, :]
+    out_1 = oracle.spectre_out(q, k, v, torch.ones(H, L // 2 + 1), H=H, F=L // 2 + 1)
+    out_s = oracle.spectre_out(q, k, v, ph, H=H, F=L // 2 + 1)
+    ref = np.roll(out_1, s, axis=1)
+    assert np.max(np.abs(out_s - ref)) < 1e-4 * np.max(np.abs(ref))
+
+
 def test_zero_gate_gives_layernorm_of_x():
     B, L, H, D = 2, 64, 2, 8
     C = H * D
