@@ -24,6 +24,7 @@ import argparse
 import glob
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -272,7 +273,11 @@ def native_arm(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps,
                              tensor_cores=False if args.cuda_core_slices else None,
-                             norm=args.norm)
+                             norm=args.norm, complex_gate=args.complex_gate)
+    if args.complex_gate:   # the workload's gate with a one-token relative phase e^{-2 pi i f / L}
+        fr = torch.arange(w.L // 2 + 1, device=dev, dtype=torch.float64)
+        d["G"] = torch.polar(d["G"].double(), -2 * math.pi * fr / w.L).to(torch.complex64)
+        d["G"] = torch.view_as_real(d["G"]).contiguous()
     h = mix.handle
 
     def barrier():
@@ -336,6 +341,7 @@ def native_arm(args, w, rank, world, local_rank):
 
     # ---- end-to-end through the host-buffer entry point
     pinned = {k: v.pin_memory() for k, v in inputs.items()}
+    pinned["G"] = d["G"].cpu().pin_memory()   # the gate as the plan reads it (real, or (re, im))
     y_host = torch.empty_like(pinned["x"]).pin_memory()
     for _ in range(2):
         binding.spectre_mix_run_host(h, pinned["q"], pinned["k"], pinned["v"], pinned["x"],
@@ -355,12 +361,12 @@ def native_arm(args, w, rank, world, local_rank):
     e2e_total = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev), dev)
     e2e_value = job_throughput(w.B * w.L, world, args.steps, e2e_total)
     nelem = w.B * w.L * w.C
-    h2d = 4 * nelem * w.elem_bytes + inputs["G"].numel() * 4 + 2 * w.C * 4
+    h2d = 4 * nelem * w.elem_bytes + pinned["G"].numel() * 4 + 2 * w.C * 4
     d2h = nelem * w.elem_bytes
 
     # ---- roofline of the path against measured HBM bandwidth
     peaks = load_peaks()
-    alg_bytes = w.algorithmic_bytes()
+    alg_bytes = w.algorithmic_bytes() + (w.H * w.F * 4 if args.complex_gate else 0)   # (re, im) gate
     achieved = alg_bytes / (ms_per_step * 1e-3) / 1e9
     traffic, per_kernel_traffic = ncu_traffic(w.name)
     names = ["rows_fwd", "slices", "rows_inv_ln"]
@@ -385,7 +391,8 @@ def native_arm(args, w, rank, world, local_rank):
                         "row pass with the previous chunk's slice pass on two streams",
         "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
                  "chunks": nchunks, "launches_per_step": nlaunch,
-                 "slice_pass": mix.slice_pass, "norm": args.norm},
+                 "slice_pass": mix.slice_pass, "norm": args.norm,
+                 "gate": "complex" if args.complex_gate else "real"},
     }
 
     # ---- CPU baseline (rank 0, N = 1 only)
@@ -436,6 +443,8 @@ def main():
     ap.add_argument("--norm", choices=["post_ln", "pre_ln", "post_rms", "pre_rms"], default="post_ln",
                     help="normalisation: LayerNorm(out + x) (default), LayerNorm(out) + x, or the "
                          "RMSNorm forms")
+    ap.add_argument("--complex-gate", action="store_true",
+                    help="time a complex gate (the workload's G with a relative-position phase)")
     ap.add_argument("--cuda-core-slices", action="store_true",
                     help="force the CUDA-core slice pass (plan option; default: tensor cores "
                          "where the plan allows)")

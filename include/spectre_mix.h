@@ -185,7 +185,14 @@ enum spectre_option {
      * SPECTRE_NORM_POST_LN, the walk-through's §2.2 form).  The other values
      * are the §3.3 variants.  The no-allocation entry point always uses the
      * default. */
-    SPECTRE_OPT_NORM = 2
+    SPECTRE_OPT_NORM = 2,
+    /* 0 (default): G is real, [H][L/2+1] fp32.  1: G is complex, a gate with
+     * a relative-position phase (walk-through §2.4): [H][L/2+1][2] fp32 as
+     * (re, im) pairs, 16-byte aligned like every tensor.  Bins above L/2 use
+     * conj(G[L - f]), so the output stays real; the imaginary parts at DC
+     * and Nyquist are dropped, as an inverse real FFT does.  The
+     * no-allocation entry point takes real gates only. */
+    SPECTRE_OPT_COMPLEX_GATE = 3
 };
 
 enum spectre_norm {

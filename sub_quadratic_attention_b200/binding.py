@@ -28,6 +28,7 @@ SPECTRE_ERR_TIMEOUT = -8
 
 SPECTRE_OPT_TENSOR_CORES = 1
 SPECTRE_OPT_NORM = 2
+SPECTRE_OPT_COMPLEX_GATE = 3
 
 # enum spectre_norm, keyed as in the oracle
 SPECTRE_NORM = {"post_ln": 0, "pre_ln": 1, "post_rms": 2, "pre_rms": 3}
@@ -211,7 +212,7 @@ class SpectreMix:
 
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
                  dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None,
-                 norm: Optional[str] = None):
+                 norm: Optional[str] = None, complex_gate: bool = False):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
         self.F = L // 2 + 1 if F is None else F
@@ -222,12 +223,32 @@ class SpectreMix:
             spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1 if tensor_cores else 0)
         if norm is not None:           # None keeps the default, "post_ln": LayerNorm(out + x)
             spectre_mix_set_option(self.handle, SPECTRE_OPT_NORM, SPECTRE_NORM[norm])
+        self.complex_gate = complex_gate
+        if complex_gate:               # G: complex [H, L/2+1] (a relative-position phase)
+            spectre_mix_set_option(self.handle, SPECTRE_OPT_COMPLEX_GATE, 1)
+        self._gate_ref = None
+
+    def _gate(self, G):
+        """G as the library reads it: a real gate as given, a complex one as its
+        (re, im) fp32 pairs.  The converted tensor stays referenced until the
+        next call, since runs are asynchronous."""
+        if G.is_complex():
+            if not self.complex_gate:
+                raise ValueError("a complex G needs a plan made with complex_gate=True")
+            import torch
+
+            G = torch.view_as_real(G.to(torch.complex64)).contiguous()
+        elif self.complex_gate:
+            raise ValueError("this plan expects a complex G")
+        self._gate_ref = G
+        return G
 
     def __call__(self, q, k, v, x, G, gamma, beta, y=None, out=None, stream=None):
         import torch
 
         if y is None:
             y = torch.empty_like(x)
+        G = self._gate(G)
         if out is None:
             spectre_mix_run(self.handle, q, k, v, x, G, gamma, beta, y, stream)
         else:
@@ -235,6 +256,7 @@ class SpectreMix:
         return y
 
     def run_host(self, q, k, v, x, G, gamma, beta, y, stream=None):
+        G = self._gate(G)
         spectre_mix_run_host(self.handle, q, k, v, x, G, gamma, beta, y, stream)
         return y
 

@@ -27,6 +27,7 @@ struct PathGeom {
     int inv_reg;         // register-resident LayerNorm variant
     int tc_mode;         // option: slice pass on the tensor cores where mma_ok (1) or CUDA cores (0)
     int norm_mode;       // option: enum spectre_norm
+    int cgate;           // option: complex gate
     int mma_ok;          // the DFT-64 MMA slice pass applies (M = 4096, fp16 P, few live groups)
     int nsm;             // multiprocessors of the device
     int chunk;           // channels per pipeline chunk (multiple of 64, or C)
@@ -196,6 +197,7 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     }
     g->tc_mode = 1;
     g->norm_mode = SPECTRE_NORM_POST_LN;
+    g->cgate = 0;
     g->nsm = 148;
     // pipeline chunks: four channel chunks when each still fills the GPU
     g->chunk = C;
@@ -277,6 +279,7 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
             sa.w64op = bf.w64op;
             sa.err = bf.err;
             sa.nbins = g.L / 2 + 1;
+            sa.cgate = g.cgate;
             sa.nslices = (long long)g.B * Cw * g.NF;
             sa.invL = 1.0f / (float)g.L;
             e = mark(st);
@@ -525,10 +528,15 @@ int spectre_mix_run_host(spectre_mix_t h, const void *q, const void *k, const vo
     const PathGeom &g = h->g;
     const size_t es = g.dtype == SPECTRE_F32 ? 4 : 2;
     const size_t nt = (size_t)g.B * g.L * g.C * es;
-    const size_t ng = (size_t)g.H * (g.L / 2 + 1) * sizeof(float);
+    const size_t ng = (size_t)g.H * (g.L / 2 + 1) * sizeof(float) * (g.cgate ? 2 : 1);
     const size_t nc = (size_t)g.C * sizeof(float);
     const size_t o_t = align_up(nt, 256), o_g = align_up(ng, 256), o_c = align_up(nc, 256);
     const size_t need = 5 * o_t + o_g + 2 * o_c;
+    if (h->stage && h->stage_bytes < need) {   // the gate grew (complex-gate option)
+        cudaFree(h->stage);
+        h->stage = nullptr;
+        h->stage_bytes = 0;
+    }
     if (!h->stage) {
         cudaError_t e = cudaMalloc(&h->stage, need);
         if (e != cudaSuccess) {
@@ -657,6 +665,10 @@ int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     case SPECTRE_OPT_TENSOR_CORES:
         if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
         h->g.tc_mode = value;
+        return SPECTRE_OK;
+    case SPECTRE_OPT_COMPLEX_GATE:
+        if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
+        h->g.cgate = value;
         return SPECTRE_OK;
     case SPECTRE_OPT_NORM:
         if (value < SPECTRE_NORM_POST_LN || value > SPECTRE_NORM_PRE_RMS) return SPECTRE_ERR_ARG;

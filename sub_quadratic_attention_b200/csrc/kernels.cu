@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     ps.smax = &smax[sl];
     ps.live = live;
     ps.p16 = a.p16 != 0;
-    const float *Gh = a.G + (size_t)h * a.nbins;
+    const float *Gh = a.G + (size_t)h * a.nbins * (a.cgate ? 2 : 1);
     __syncthreads();  // smax initialised
 
     float2 x[RL];
@@ -517,8 +517,15 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     for (int r = 0; r < RL; r++) {
         int f = f1 + a.R * (j + r * NT);
         int ff = min(f, a.L - f);
-        float g = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
-        put(r, cscale(x[r], g));
+        if (a.cgate) {   // conj(G[L - f]) above L/2
+            float2 gc = (live && ff < a.F) ? __ldg(reinterpret_cast<const float2 *>(Gh) + ff)
+                                           : make_float2(0.f, 0.f);
+            if (f > a.L - f) gc.y = -gc.y;
+            put(r, cscale(cmul(x[r], gc), a.invL));
+        } else {
+            float g = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
+            put(r, cscale(x[r], g));
+        }
     }
     if constexpr (Cfg::NP >= 2) __syncthreads();
     // k: S *= conj(K)

@@ -55,7 +55,8 @@ struct SliceArgs {
     void *P;              // float2 [B][C][NF][M], or __half2 pair-interleaved (p16_pair_slice)
     float *pscale;        // p16: P = stored * pscale, pair-interleaved like P
     const float2 *twL;
-    const float *G;       // [H][L/2+1]
+    const float *G;       // [H][L/2+1], or with cgate [H][L/2+1][2] (re, im)
+    int cgate;            // complex gate: conj(G[L - f]) above L/2
     SliceTables tabs;
     int B, L, R, M, C, D, F, nbins;
     int c_lo, Cw;         // channel wave

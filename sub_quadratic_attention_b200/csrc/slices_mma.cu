@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
         const int b = (int)(rest / npair);
         const int c = a.c_lo + cl;
         const bool live = cl < a.Cw && c < a.C;
-        const float *Gh = a.G + (size_t)(live ? c / a.D : 0) * a.nbins;
+        const float *Gh = a.G + (size_t)(live ? c / a.D : 0) * a.nbins * (a.cgate ? 2 : 1);
         const float2 *srcA = a.A + ((size_t)(b * a.Cw + (live ? cl : 0)) * NF + f1) * kM;
 
         // k2 groups (8 k2 values) that hold a bin with a nonzero gate
@@ -330,8 +330,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSM) spectre_slices_mma4096
                         if (sig == 0) {
                             const int f = f1 + a.R * (row + 64 * (8 * g + j));
                             const int ff = min(f, a.L - f);
-                            const float gate = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
-                            S = cscale(X, gate);
+                            if (a.cgate) {   // conj(G[L - f]) above L/2
+                                float2 gc = (live && ff < a.F)
+                                                ? __ldg(reinterpret_cast<const float2 *>(Gh) + ff)
+                                                : make_float2(0.f, 0.f);
+                                if (f > a.L - f) gc.y = -gc.y;
+                                S = cscale(cmul(X, gc), a.invL);
+                            } else {
+                                const float gate = (live && ff < a.F) ? __ldg(Gh + ff) * a.invL : 0.f;
+                                S = cscale(X, gate);
+                            }
                         } else if (sig == 1) {
                             S = cmulc(make_float2(sv[2 * j], sv[2 * j + 1]), X);
                         } else {

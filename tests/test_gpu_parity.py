@@ -183,3 +183,27 @@ def test_norm_variants(norm, case):
     out_ref, y_ref = oracle_full(w, inp, norm=norm)
     e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
     print(f"{norm} {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+def _complex_gate(G, seed):
+    """G with a seeded phase in (-pi, pi] per bin: a complex64 gate."""
+    th = (torch.rand(G.shape, generator=torch.Generator().manual_seed(seed)) * 2 - 1) * np.pi
+    return torch.polar(G.float(), th.float())
+
+
+@pytest.mark.parametrize("case", ["bf16_long", "fp32_mid", (2, 12288, 2, 8, 6145),
+                                  (1, 524288, 1, 4, 5000)])
+def test_complex_gate(case):
+    """A complex gate (relative-position phase) in both slice passes: the
+    tensor-core one (bf16_long), the CUDA-core one in fp32 and in bf16 with a
+    mixed-radix length, and R = 64."""
+    if isinstance(case, str):
+        w = WORKLOADS[case]
+    else:
+        w = custom(*case, dtype="bf16" if case[1] == 12288 else "f32")
+    inp = make_inputs(w)
+    inp["G"] = _complex_gate(inp["G"], seed=w.L)
+    out, y = run_library(w, inp, complex_gate=True)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"complex gate {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
