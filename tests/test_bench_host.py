@@ -1,0 +1,52 @@
+"""Host-side logic of bench.py that needs no GPU: the code-only source hash that
+keys the stored ncu traffic, and the lookup of that traffic."""
+import os
+import shutil
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_code_only_drops_comments_and_whitespace_but_keeps_code():
+    a = "int f(int x) {  // twice\n    return 2 * x; /* the\n double */\n}\n"
+    b = "int f(int x) { return 2 * x; }"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(b.replace("2", "3"))
+    # comment markers inside literals are code
+    s = 'const char *u = "http://x"; char c = \'/\';'
+    assert "http://x" in bench._code_only(s)
+
+
+def _copy_sources(dst):
+    for sub in ("sub_quadratic_attention_b200/csrc", "include"):
+        shutil.copytree(os.path.join(ROOT, sub), os.path.join(dst, sub))
+
+
+def test_source_hash_ignores_a_comment_edit_and_sees_a_code_edit(tmp_path, monkeypatch):
+    _copy_sources(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.source_hash()
+    f = tmp_path / "sub_quadratic_attention_b200" / "csrc" / "api.cu"
+    text = f.read_text()
+    f.write_text("// an added comment line\n" + text)
+    assert bench.source_hash() == h0
+    f.write_text(text.replace("return SPECTRE_OK;", "return SPECTRE_OK; ", 1) + "\nstatic int extra;\n")
+    assert bench.source_hash() != h0
+
+
+def test_traffic_is_used_only_under_its_source_hash(tmp_path, monkeypatch):
+    _copy_sources(tmp_path)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_hash()
+    lines = ["# workload source_hash kernel dram_bytes_per_step",
+             f"wl {h} rows_fwd 100", f"wl {h} slices 200", f"wl {h} rows_inv_ln 50",
+             "wl 000000000000 rows_fwd 999", f"part {h} rows_fwd 1"]
+    (tmp_path / "profiles" / "traffic.txt").write_text("\n".join(lines) + "\n")
+    total, per = bench.ncu_traffic("wl")
+    assert total == 350 and per == {"rows_fwd": 100.0, "slices": 200.0, "rows_inv_ln": 50.0}
+    assert bench.ncu_traffic("other")[0] is None
+    assert bench.ncu_traffic("part")[0] is None    # only a complete step counts
