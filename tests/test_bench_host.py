@@ -50,3 +50,21 @@ def test_traffic_is_used_only_under_its_source_hash(tmp_path, monkeypatch):
     assert total == 350 and per == {"rows_fwd": 100.0, "slices": 200.0, "rows_inv_ln": 50.0}
     assert bench.ncu_traffic("other")[0] is None
     assert bench.ncu_traffic("part")[0] is None    # only a complete step counts
+
+
+def test_dominant_kernel_roofline_arithmetic():
+    """bf16 long's figures: 335.81 MB of algorithmic bytes over B L C =
+    33,554,432 elements (10.008 B each); the slice pass is dominant with two
+    launches in 0.2 ms per step, so a launch moves half the elements'
+    bytes in 0.1 ms."""
+    names = ["rows_fwd", "slices", "rows_inv_ln"]
+    r = bench.dominant_roofline(335_810_560, 33_554_432, [0.1378, 0.2000, 0.0846], [2, 2, 1],
+                                {"slices": 527_414_272.0}, names, 6554.6)
+    assert r["kernel"] == "slices" and r["units_per_launch"] == 16_777_216
+    assert abs(r["bytes_per_unit"] - 10.0079) < 1e-3
+    assert abs(r["launch_ms"] - 0.1) < 1e-9
+    assert abs(r["achieved"] - 335.81056 / 0.2) < 0.01          # GB/s
+    assert abs(r["frac"] - (335.81056 / 0.2) / 6554.6) < 1e-4
+    assert r["traffic"] == 527_414_272.0 / 2
+    r2 = bench.dominant_roofline(100.0, 10, [1.0, 0.5, 3.0], [2, 2, 1], {}, names, 1000.0)
+    assert r2["kernel"] == "rows_inv_ln" and r2["traffic"] is None
