@@ -271,12 +271,36 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(w, world):
-    return {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "C": w.C, "F": w.F,
-            "io_dtype": w.dtype, "global_batch": w.B * world, "seq_len": w.L,
-            "parallelism": f"dp{world} (independent batch per rank, no data-path collective)",
-            "l2": "flushed before every timed step (256 MiB memset, outside the timed interval); "
-                  "inputs 268 MB also exceed L2"}
+def config_dict(w, world, pw=None):
+    cfg = {"workload": w.name, "B": w.B, "L": w.L, "H": w.H, "D": w.D, "C": w.C, "F": w.F,
+           "io_dtype": w.dtype, "global_batch": w.B * world, "seq_len": w.L,
+           "parallelism": f"dp{world} (independent batch per rank, no data-path collective)",
+           "l2": "flushed before every timed step (256 MiB memset, outside the timed interval); "
+                 "inputs 268 MB also exceed L2"}
+    if pw is not None and pw is not w:
+        cfg.update({"workload": pw.name, "block_len": pw.L, "F": pw.F,
+                    "mode": f"blockwise: the mix within each block of {pw.L} tokens "
+                            f"({w.B * w.L // pw.L} blocks), gate [H, {pw.L // 2 + 1}]"})
+    return cfg
+
+
+def block_view(w, inputs, n):
+    """Blockwise mode's plan shape and inputs: the workload's q, k, v, x viewed
+    as B L / n sequences of n tokens (same memory), the first n/2 + 1 bins of
+    its gate, and F scaled by n / L (the same fraction of bins kept)."""
+    from sub_quadratic_attention_b200.workloads import custom
+
+    if n < 2 or w.L % n:
+        raise SystemExit(f"--block-len must divide L = {w.L}")
+    F = max(1, min(n // 2 + 1, w.F * n // w.L))
+    pw = custom(w.B * (w.L // n), n, w.H, w.D, F, dtype=w.dtype, qkv_scale=w.qkv_scale,
+                x_scale=w.x_scale, gate=w.gate, gamma=w.gamma, beta=w.beta,
+                name=f"{w.name}_block{n}", index=w.index)
+    shape = (pw.B, pw.L, pw.C)
+    out = {k: inputs[k].view(shape) for k in ("q", "k", "v", "x")}
+    out.update(G=inputs["G"][:, :n // 2 + 1].contiguous(), gamma=inputs["gamma"],
+               beta=inputs["beta"])
+    return pw, out
 
 
 # ---------------------------------------------------------------------------
@@ -293,16 +317,20 @@ def native_arm(args, w, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     inputs = make_inputs(w, seed_offset=rank_seed_offset(rank))
+    pw = w          # the shape the plan runs: w itself, or its blocks in blockwise mode
+    if args.block_len:
+        pw, inputs = block_view(w, inputs, args.block_len)
     d = {k: v.to(dev) for k, v in inputs.items()}
     y = torch.empty_like(d["x"])
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    mix = binding.SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps,
+    mix = binding.SpectreMix(w.B, w.L, w.H, w.D, pw.F, w.dtype, w.eps,
                              tensor_cores=False if args.cuda_core_slices else None,
-                             norm=args.norm, complex_gate=args.complex_gate)
+                             norm=args.norm, complex_gate=args.complex_gate,
+                             block_len=args.block_len or None)
     if args.complex_gate:   # the workload's gate with a one-token relative phase e^{-2 pi i f / L}
-        fr = torch.arange(w.L // 2 + 1, device=dev, dtype=torch.float64)
-        d["G"] = torch.polar(d["G"].double(), -2 * math.pi * fr / w.L).to(torch.complex64)
+        fr = torch.arange(pw.L // 2 + 1, device=dev, dtype=torch.float64)
+        d["G"] = torch.polar(d["G"].double(), -2 * math.pi * fr / pw.L).to(torch.complex64)
         d["G"] = torch.view_as_real(d["G"]).contiguous()
     h = mix.handle
 
@@ -392,9 +420,9 @@ def native_arm(args, w, rank, world, local_rank):
 
     # ---- roofline of the path against measured HBM bandwidth
     peaks = load_peaks()
-    alg_bytes = w.algorithmic_bytes() + (w.H * w.F * 4 if args.complex_gate else 0)   # (re, im) gate
+    alg_bytes = pw.algorithmic_bytes() + (w.H * pw.F * 4 if args.complex_gate else 0)   # (re, im) gate
     achieved = alg_bytes / (ms_per_step * 1e-3) / 1e9
-    traffic, per_kernel_traffic = ncu_traffic(w.name)
+    traffic, per_kernel_traffic = ncu_traffic(pw.name)
     names = ["rows_fwd", "slices", "rows_inv_ln"]
     kmean = [sum(k) / len(k) for k in kern_ms]
     ksum = sum(kmean)
@@ -423,13 +451,14 @@ def native_arm(args, w, rank, world, local_rank):
         "plan": {"R": R, "M": M, "slices_per_channel": nf, "channels_per_wave": wave_ch,
                  "chunks": nchunks, "launches_per_step": nlaunch,
                  "slice_pass": mix.slice_pass, "norm": args.norm,
-                 "gate": "complex" if args.complex_gate else "real"},
+                 "gate": "complex" if args.complex_gate else "real",
+                 "block_len": args.block_len or None},
     })
 
     # ---- CPU baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, nch, nthreads = time_oracle_sample(w, inputs, args.cpu_seconds)
+        rate, dt, nch, nthreads = time_oracle_sample(pw, inputs, args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                "sample": f"oracle (fp64) on channels 0..{nch - 1} of {w.C}, all {w.B * w.L} "
                          f"tokens, pre-LayerNorm output, {dt:.1f} s; tokens/s scaled by "
@@ -449,7 +478,7 @@ def native_arm(args, w, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; shapes and distributions of the bf16 long workload)",
-            "config": config_dict(w, world),
+            "config": config_dict(w, world, pw),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": nlaunch * args.steps,
@@ -476,6 +505,8 @@ def main():
                          "RMSNorm forms")
     ap.add_argument("--complex-gate", action="store_true",
                     help="time a complex gate (the workload's G with a relative-position phase)")
+    ap.add_argument("--block-len", type=int, default=0,
+                    help="blockwise mode: mix within blocks of this many tokens (must divide L)")
     ap.add_argument("--cuda-core-slices", action="store_true",
                     help="force the CUDA-core slice pass (plan option; default: tensor cores "
                          "where the plan allows)")

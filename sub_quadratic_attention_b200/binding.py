@@ -203,22 +203,57 @@ def spectre_mix_plan_info(h: int) -> Tuple[int, int, int, int, int]:
     return tuple(v.value for v in vals)
 
 
+def check_arguments(B, L, H, C, plan_L, dtype_code, q, k, v, x, G, gamma, beta, y, out=None):
+    """Sizes and element types of one run's tensors, checked on the host: the
+    library reads raw pointers, so a short buffer would be read out of bounds.
+    q, k, v, x, y hold B * L * C values of the plan's type (bf16 or fp32); G
+    holds H * (plan_L / 2 + 1) fp32 values (complex64 for a complex gate);
+    gamma, beta hold C fp32 values; out (optional) B * L * C fp32 values."""
+    import torch
+
+    n = B * L * C
+    tok_type = torch.float32 if dtype_code == SPECTRE_F32 else torch.bfloat16
+    for name, t in (("q", q), ("k", k), ("v", v), ("x", x), ("y", y)):
+        if t.numel() != n or t.dtype != tok_type:
+            raise ValueError(f"{name} must hold B * L * C = {n} values of {tok_type}")
+    if out is not None and (out.numel() != n or out.dtype != torch.float32):
+        raise ValueError(f"out must hold B * L * C = {n} fp32 values")
+    nb = plan_L // 2 + 1
+    if G.numel() != H * nb or G.dtype not in (torch.float32, torch.complex64, torch.complex128):
+        raise ValueError(f"G must be [H, {nb}], fp32 (or complex for a complex gate)")
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if t.numel() != C or t.dtype != torch.float32:
+            raise ValueError(f"{name} must hold C = {C} fp32 values")
+
+
 class SpectreMix:
     """A plan for one shape, usable with torch CUDA tensors.
 
     ``mix(q, k, v, x, G, gamma, beta)`` returns y; pass ``out=`` (fp32
     [B, L, C]) to also receive the pre-LayerNorm mixer output.
+
+    ``block_len``: blockwise mode (walk-through §3.2, ``fft_len``): the mix runs
+    within each block of block_len consecutive tokens, as B * L / block_len
+    independent sequences of length block_len.  A [B, L, C] tensor is already
+    laid out as [B * L / block_len, block_len, C], so only the plan's shape
+    changes; G is then [H, block_len / 2 + 1] and F counts the block's bins.
+    (The pages leave the exchange between blocks unspecified; none is done.)
     """
 
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
                  dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None,
-                 norm: Optional[str] = None, complex_gate: bool = False):
+                 norm: Optional[str] = None, complex_gate: bool = False,
+                 block_len: Optional[int] = None):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
-        self.F = L // 2 + 1 if F is None else F
+        if block_len is not None and (block_len < 1 or L % block_len):
+            raise ValueError("block_len must divide L")
+        self.block_len = block_len
+        self.plan_B, self.plan_L = (B * (L // block_len), block_len) if block_len else (B, L)
+        self.F = self.plan_L // 2 + 1 if F is None else F
         self.dtype_code = SPECTRE_F32 if dtype in ("f32", "float32", "fp32") else SPECTRE_BF16
         self.eps = eps
-        self.handle = spectre_mix_create(B, L, H, D, self.F, self.dtype_code, eps)
+        self.handle = spectre_mix_create(self.plan_B, self.plan_L, H, D, self.F, self.dtype_code, eps)
         if tensor_cores is not None:   # None keeps the library's default (on)
             spectre_mix_set_option(self.handle, SPECTRE_OPT_TENSOR_CORES, 1 if tensor_cores else 0)
         if norm is not None:           # None keeps the default, "post_ln": LayerNorm(out + x)
@@ -227,6 +262,10 @@ class SpectreMix:
         if complex_gate:               # G: complex [H, L/2+1] (a relative-position phase)
             spectre_mix_set_option(self.handle, SPECTRE_OPT_COMPLEX_GATE, 1)
         self._gate_ref = None
+
+    def _check_shapes(self, q, k, v, x, G, gamma, beta, y, out):
+        check_arguments(self.B, self.L, self.H, self.C, self.plan_L, self.dtype_code,
+                        q, k, v, x, G, gamma, beta, y, out)
 
     def _gate(self, G):
         """G as the library reads it: a real gate as given, a complex one as its
@@ -248,6 +287,7 @@ class SpectreMix:
 
         if y is None:
             y = torch.empty_like(x)
+        self._check_shapes(q, k, v, x, G, gamma, beta, y, out)
         G = self._gate(G)
         if out is None:
             spectre_mix_run(self.handle, q, k, v, x, G, gamma, beta, y, stream)
@@ -256,6 +296,7 @@ class SpectreMix:
         return y
 
     def run_host(self, q, k, v, x, G, gamma, beta, y, stream=None):
+        self._check_shapes(q, k, v, x, G, gamma, beta, y, None)
         G = self._gate(G)
         spectre_mix_run_host(self.handle, q, k, v, x, G, gamma, beta, y, stream)
         return y

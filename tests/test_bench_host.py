@@ -68,3 +68,24 @@ def test_dominant_kernel_roofline_arithmetic():
     assert r["traffic"] == 527_414_272.0 / 2
     r2 = bench.dominant_roofline(100.0, 10, [1.0, 0.5, 3.0], [2, 2, 1], {}, names, 1000.0)
     assert r2["kernel"] == "rows_inv_ln" and r2["traffic"] is None
+
+
+def test_block_view_keeps_memory_and_scales_F():
+    import torch
+
+    from sub_quadratic_attention_b200.workloads import custom, make_inputs
+
+    w = custom(2, 256, 2, 4, 65, dtype="bf16")
+    inp = make_inputs(w)
+    pw, b = bench.block_view(w, inp, 64)
+    assert (pw.B, pw.L, pw.C, pw.F) == (8, 64, 8, 16)        # F keeps the fraction 65/256 of L
+    for k in ("q", "k", "v", "x"):
+        assert b[k].shape == (8, 64, 8) and b[k].data_ptr() == inp[k].data_ptr()
+    assert torch.equal(b["G"], inp["G"][:, :33]) and b["G"].is_contiguous()
+    assert pw.algorithmic_bytes() == 5 * 2 * 256 * 8 * 2 + 2 * 16 * 4 + 2 * 8 * 4
+    cfg = bench.config_dict(w, 1, pw)
+    assert cfg["block_len"] == 64 and cfg["L"] == 256 and cfg["F"] == 16
+    import pytest
+
+    with pytest.raises(SystemExit):
+        bench.block_view(w, inp, 100)

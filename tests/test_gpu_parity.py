@@ -207,3 +207,35 @@ def test_complex_gate(case):
     out_ref, y_ref = oracle_full(w, inp)
     e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
     print(f"complex gate {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+@pytest.mark.parametrize("B,L,H,D,n,F,dtype", [
+    (2, 16384, 4, 32, 4096, 1000, "bf16"),
+    (1, 131072, 2, 32, 65536, 8192, "bf16"),     # tensor-core slice pass inside each block
+    (1, 3 * 12288, 2, 8, 12288, 6145, "f32"),    # mixed-radix blocks
+    (3, 1024, 1, 16, 256, 129, "f32"),
+    (1, 4096, 2, 16, 4096, 2049, "f32"),         # one block: the plain mix
+])
+def test_blockwise_mode(B, L, H, D, n, F, dtype):
+    """Blockwise mode: the library, planned on [B, L, C] with block_len = n,
+    against the oracle run on the same values as B L / n sequences of n
+    tokens with the block's gate [H, n/2 + 1]."""
+    from sub_quadratic_attention_b200 import binding
+    from sub_quadratic_attention_b200.binding import SpectreMix
+
+    wb = custom(B * (L // n), n, H, D, F, dtype=dtype)
+    inp = make_inputs(wb)
+    C = H * D
+    d = {k: t.cuda() for k, t in inp.items()}
+    with SpectreMix(B, L, H, D, F, dtype, wb.eps, block_len=n) as mix:
+        y = torch.empty((B, L, C), dtype=d["x"].dtype, device="cuda")
+        out = torch.empty((B, L, C), dtype=torch.float32, device="cuda")
+        mix(d["q"].view(B, L, C), d["k"].view(B, L, C), d["v"].view(B, L, C),
+            d["x"].view(B, L, C), d["G"], d["gamma"], d["beta"], y=y, out=out)
+        torch.cuda.synchronize()
+        assert binding.spectre_mix_device_status(mix.handle) == binding.SPECTRE_OK
+        assert mix.slice_pass == _expected_slice_pass(wb)
+    out_ref, y_ref = oracle_full(wb, inp)
+    e_out, e_y = check_parity(wb, out.cpu().view(wb.B, n, C), y.cpu().view(wb.B, n, C),
+                              out_ref, y_ref)
+    print(f"block mode {B}x{L} n={n}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
