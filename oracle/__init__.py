@@ -1,16 +1,22 @@
-"""Double-precision CPU oracle for SPECTRE frequency-domain token mixing.
+"""Double-precision CPU oracles: SPECTRE frequency-domain token mixing, and
+per-token DCT mixing with spectral-entropy routing.
 
 TEST INFRASTRUCTURE ONLY.  The test suite, the smoke check and the CPU-baseline
 leg of ``bench.py`` are the only callers.  The CUDA library never imports,
 links or calls anything here, and nothing here imports the CUDA library.
 
-The arithmetic lives in ``spectre_oracle.c`` (plain C, fp64, OpenMP over
-channels).  This module only marshals arrays through ctypes.
+The arithmetic lives in ``spectre_oracle.c`` and ``dct_oracle.c`` (plain C,
+fp64, OpenMP over channels or tokens).  This module only marshals arrays
+through ctypes.
 
 What the oracle computes follows the SPECTRE walk-through
 (hotelren.com/news/5925787): §2.2 pseudocode (FFT of q, k, v along the
 sequence, ``Q_f * conj(K_f)`` gated by ``G``, times ``V_f``, inverse FFT,
 ``layer_norm(out + x)``) and §2.3 (keep only the low-frequency bins f < F).
+The DCT mix follows the Chiaroscuro Attention summary
+(paper.rainbus.top/paper/2606.08327): the orthonormal Type-II DCT of each
+token, its normalised spectral entropy H(x), the routing rule H(x) <= tau,
+and DCTMix without its feed-forward layer, LayerNorm(x + iDCT(DCT(x) * w)).
 """
 from __future__ import annotations
 
@@ -22,16 +28,17 @@ from typing import Optional, Sequence
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "spectre_oracle.c")
+_SRCS = [os.path.join(_HERE, "spectre_oracle.c"), os.path.join(_HERE, "dct_oracle.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``spectre_oracle.c`` into ``liboracle.so`` beside it."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-Wall", "-o", _LIB, _SRC, "-lm"]
+    """Compile the oracle's C sources into ``liboracle.so`` beside them."""
+    newest = max(os.path.getmtime(s) for s in _SRCS)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-Wall", "-o", _LIB, *_SRCS, "-lm"]
         subprocess.check_call(cmd)
     return _LIB
 
@@ -54,6 +61,13 @@ def _load():
             ctypes.c_double, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_long, vp, vp, ctypes.c_int,
             ctypes.c_int, ctypes.c_int]
         lib.oracle_spectre_mix.restype = ctypes.c_int
+        for name in ("oracle_dct2", "oracle_dct3"):
+            getattr(lib, name).argtypes = [ctypes.c_long, ctypes.c_long, vp, vp]
+            getattr(lib, name).restype = ctypes.c_int
+        lib.oracle_dct_mix.argtypes = [
+            ctypes.c_long, ctypes.c_long, ctypes.c_int, vp, vp, vp, vp, ctypes.c_double,
+            ctypes.c_double, vp, vp, vp, vp, ctypes.c_int]
+        lib.oracle_dct_mix.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -182,3 +196,61 @@ def spectre_mix(q, k, v, x, G, gamma, beta, H: int, F: int, eps: float = 1e-5,
     if rc != 0:
         raise RuntimeError("oracle_spectre_mix failed")
     return out, y
+
+
+# ---------------------------------------------------------------------------
+# per-token DCT mixing (Chiaroscuro Attention summary)
+# ---------------------------------------------------------------------------
+def _rows64(a) -> np.ndarray:
+    import torch
+
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def dct2(x) -> np.ndarray:
+    """Orthonormal Type-II DCT along the last axis ("Prerequisites: DCT")."""
+    a = _rows64(x)
+    d = a.shape[-1]
+    out = np.empty_like(a)
+    if _load().oracle_dct2(a.size // d, d, _ptr(a), _ptr(out)) != 0:
+        raise RuntimeError("oracle_dct2 failed")
+    return out
+
+
+def idct2(X) -> np.ndarray:
+    """Inverse of ``dct2`` (the orthonormal Type-III DCT) along the last axis."""
+    a = _rows64(X)
+    d = a.shape[-1]
+    out = np.empty_like(a)
+    if _load().oracle_dct3(a.size // d, d, _ptr(a), _ptr(out)) != 0:
+        raise RuntimeError("oracle_dct3 failed")
+    return out
+
+
+def dct_mix(x, w, gamma, beta, eps: float = 1e-5, tau: float = 0.8954, nthreads: int = 0):
+    """The DCT mix of token rows ``x[..., d]`` (fp32 or bf16, widened exactly).
+
+    Returns a dict of float64 ``mix`` (iDCT(DCT(x) * w), before the residual),
+    ``y`` (LayerNorm_d(x + mix; gamma, beta, eps)), ``H`` (normalised spectral
+    entropy per token) and uint8 ``route`` (1 where H <= tau).  ``eps`` and
+    ``tau`` are taken as the fp32 values the library receives.
+    """
+    xa, dt = _as_stored(x)
+    shape = xa.shape
+    d = shape[-1]
+    T = xa.size // d
+    mix = np.empty(shape, dtype=np.float64)
+    y = np.empty(shape, dtype=np.float64)
+    H = np.empty(shape[:-1], dtype=np.float64)
+    route = np.empty(shape[:-1], dtype=np.uint8)
+    wa, ga, ba = _f32(w), _f32(gamma), _f32(beta)
+    if wa.size != d or ga.size != d or ba.size != d:
+        raise ValueError("w, gamma and beta must hold d values")
+    rc = _load().oracle_dct_mix(T, d, dt, _ptr(xa), _ptr(wa), _ptr(ga), _ptr(ba),
+                                float(np.float32(eps)), float(np.float32(tau)), _ptr(mix),
+                                _ptr(y), _ptr(H), _ptr(route), nthreads)
+    if rc != 0:
+        raise RuntimeError("oracle_dct_mix failed")
+    return {"mix": mix, "y": y, "H": H, "route": route}
