@@ -17,6 +17,10 @@ q, k, v, x, G, gamma, beta from pinned memory, the mix, and the D2H copy of y.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
 same workload (rank 0 only).
+
+``--workload dct_d256`` or ``dct_d1024`` times the per-token DCT mix with
+spectral-entropy routing instead (x [B, L, d] bf16, one kernel per step), with
+the same L2 flush, timing, e2e, roofline, clocks and CPU-oracle legs.
 """
 from __future__ import annotations
 
@@ -76,12 +80,19 @@ def _code_only(text: str) -> str:
     return " ".join("".join(out).split())
 
 
-def source_hash() -> str:
-    """Hash of the library's code (csrc/ and include/, comments and whitespace
+def source_hash(path: str = "spectre") -> str:
+    """Hash of one path's code in the library (comments and whitespace
     ignored); the ncu traffic in profiles/traffic.txt is used only under the
-    hash it was captured on."""
+    hash it was captured on.  path "spectre": csrc/ and include/ without the
+    DCT mix's files (named dct_*); path "dct": the DCT mix's files and the
+    headers they include (spectre_mix.h, fft_regs.cuh)."""
     files = sorted(glob.glob(os.path.join(ROOT, "sub_quadratic_attention_b200", "csrc", "*")) +
                    glob.glob(os.path.join(ROOT, "include", "*.h")))
+    if path == "dct":
+        files = [f for f in files if os.path.basename(f).startswith("dct_") or
+                 os.path.basename(f) in ("spectre_mix.h", "fft_regs.cuh")]
+    else:
+        files = [f for f in files if not os.path.basename(f).startswith("dct_")]
     h = hashlib.sha1()
     for f in files:
         with open(f, encoding="utf-8", errors="replace") as fh:
@@ -90,12 +101,12 @@ def source_hash() -> str:
     return h.hexdigest()[:12]
 
 
-def ncu_traffic(workload: str):
+def ncu_traffic(workload: str, path: str = "spectre", kernels: int = 3):
     """DRAM bytes per step from profiles/traffic.txt, if taken on this source."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None, {}
-    cur = source_hash()
+    cur = source_hash(path)
     per = {}
     with open(p) as f:
         for line in f:
@@ -108,7 +119,7 @@ def ncu_traffic(workload: str):
             wl, hsh, kern, nbytes = parts
             if wl == workload and hsh == cur:
                 per[kern] = float(nbytes)
-    if len(per) == 3:
+    if len(per) == kernels:
         return sum(per.values()), per
     return None, {}
 
@@ -491,6 +502,199 @@ def native_arm(args, w, rank, world, local_rank):
     mix.close()
 
 
+# ---------------------------------------------------------------------------
+# DCT mix (per-token DCT, spectral entropy, route, LayerNorm(x + iDCT(DCT(x) w)))
+# ---------------------------------------------------------------------------
+def dct_metric(w) -> str:
+    return (f"dct-mix tokens/s at B{w.B} L{w.L} d{w.d} {w.dtype}; achieved HBM GB/s vs peak")
+
+
+def dct_config(w, world):
+    return {"workload": w.name, "B": w.B, "L": w.L, "d": w.d, "tau": w.tau, "io_dtype": w.dtype,
+            "global_batch": w.B * world, "seq_len": w.L,
+            "parallelism": f"dp{world} (independent tokens per rank, no data-path collective)",
+            "l2": "flushed before every timed step (256 MiB memset, outside the timed interval); "
+                  f"x alone is {w.T * w.d * w.elem_bytes / 1e6:.0f} MB"}
+
+
+def time_dct_oracle_sample(w, inputs, target_s: float):
+    """Time the oracle on the first n token rows, growing n until one call
+    takes about target_s.  Returns (tokens per second, seconds, n, threads)."""
+    import oracle
+
+    nthreads = os.cpu_count() or 1
+    x = inputs["x"].reshape(-1, w.d)
+    n = 64
+    while True:
+        t0 = time.perf_counter()
+        oracle.dct_mix(x[:n], inputs["w"], inputs["gamma"], inputs["beta"], eps=w.eps, tau=w.tau,
+                       nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= w.T:
+            break
+        n = min(w.T, n * max(2, int(target_s / max(dt, 1e-3))))
+    return n / dt, dt, n, nthreads
+
+
+def dct_reference_arm(args, w, rank, world):
+    if rank != 0:
+        return
+    from sub_quadratic_attention_b200.workloads import make_dct_inputs
+
+    inputs = make_dct_inputs(w)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    _, _, n, nthreads = time_dct_oracle_sample(w, inputs, per_step)
+    import oracle
+
+    x = inputs["x"].reshape(-1, w.d)[:n]
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.dct_mix(x, inputs["w"], inputs["gamma"], inputs["beta"], eps=w.eps, tau=w.tau,
+                       nthreads=nthreads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    mean = sum(times) / len(times)
+    value = n / mean
+    sample = f"oracle (fp64, O(d^2) DCT sums, OpenMP) on the first {n} of {w.T} token rows"
+    print(json.dumps({
+        "impl": "reference", "metric": dct_metric(w), "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dct_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def dct_arm(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from sub_quadratic_attention_b200 import binding
+    from sub_quadratic_attention_b200.ranks import job_throughput, max_over_ranks, rank_seed_offset
+    from sub_quadratic_attention_b200.workloads import make_dct_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inputs = make_dct_inputs(w, seed_offset=rank_seed_offset(rank))
+    d = {k: v.to(dev) for k, v in inputs.items()}
+    lead = (w.B, w.L)
+    y = torch.empty_like(d["x"])
+    H = torch.empty(lead, dtype=torch.float32, device=dev)
+    route = torch.empty(lead, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    mix = binding.DctMix(w.d, w.dtype, w.eps)
+    h = mix.handle
+
+    def step():
+        binding.dct_mix_run(h, w.T, d["x"], d["w"], d["gamma"], d["beta"], w.tau, y, H, route,
+                            stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier()
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    ms_per_step = total_ms / args.steps
+    value = job_throughput(w.T, world, args.steps, total_ms)
+
+    # e2e through the host-buffer entry point
+    pinned = {k: v.pin_memory() for k, v in inputs.items()}
+    y_h = torch.empty_like(pinned["x"]).pin_memory()
+    H_h = torch.empty(lead, dtype=torch.float32).pin_memory()
+    r_h = torch.empty(lead, dtype=torch.uint8).pin_memory()
+
+    def host_step():
+        binding.dct_mix_run_host(h, w.T, pinned["x"], pinned["w"], pinned["gamma"],
+                                 pinned["beta"], w.tau, y_h, H_h, r_h, stream)
+
+    for _ in range(2):
+        host_step()
+    torch.cuda.synchronize()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        host_step()
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_total = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev), dev)
+    e2e_value = job_throughput(w.T, world, args.steps, e2e_total)
+    es = w.elem_bytes
+    h2d = w.T * w.d * es + 3 * w.d * 4
+    d2h = w.T * w.d * es + 5 * w.T
+
+    peaks = load_peaks()
+    alg = w.algorithmic_bytes()
+    achieved = alg / (ms_per_step * 1e-3) / 1e9
+    traffic, _ = ncu_traffic(w.name, path="dct", kernels=1)
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+        "kernel": "dct_mix", "bytes_per_unit": round(alg / w.T, 4), "units_per_launch": w.T,
+        "launch_ms": round(ms_per_step, 5),
+        "peak_source": f"{peaks['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+        if peaks["source"] == "measured" else "fallback 6.65 TB/s",
+        "scope": "the step's one kernel: algorithmic bytes per token (x read and y written, "
+                 "d values each, H and route written; w, gamma, beta once per launch) x the "
+                 "tokens of a launch, over its CUDA-event time",
+    }
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, n, nthreads = time_dct_oracle_sample(w, inputs, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"oracle (fp64) on the first {n} of {w.T} token rows, {dt:.1f} s"}
+    if world > 1:
+        gathered = [None] * world
+        dist.all_gather_object(gathered, clocks)
+        clocks = dict(clocks)
+        clocks["reasons"] = sorted({r for c in gathered for r in c.get("reasons", [])})
+    if rank == 0:
+        print(json.dumps({
+            "metric": dct_metric(w), "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": f"synthetic (seeded; half smooth, half white token rows, d = {w.d})",
+            "config": dct_config(w, world),
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "routed_fraction": round(float(route.float().mean().item()), 4),
+            "hbm_gbs_achieved": round(achieved, 2),
+        }), flush=True)
+    mix.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,11 +727,14 @@ def main():
                   flush=True)
             sys.exit(2)
 
-    from sub_quadratic_attention_b200.workloads import WORKLOADS
+    from sub_quadratic_attention_b200.workloads import DCT_WORKLOADS, WORKLOADS
 
-    w = WORKLOADS[args.workload]
+    dct = args.workload in DCT_WORKLOADS
+    if not dct and args.workload not in WORKLOADS:
+        ap.error(f"unknown workload {args.workload}")
+    w = DCT_WORKLOADS[args.workload] if dct else WORKLOADS[args.workload]
     if args.impl == "reference":
-        reference_arm(args, w, rank, world)
+        (dct_reference_arm if dct else reference_arm)(args, w, rank, world)
         return
     if world > 1:
         import datetime
@@ -539,7 +746,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        native_arm(args, w, rank, world, local_rank)
+        (dct_arm if dct else native_arm)(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

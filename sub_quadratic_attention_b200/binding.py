@@ -1,8 +1,9 @@
-"""ctypes binding of libspectre_mix (C ABI in include/spectre_mix.h).
+"""ctypes binding of libspectre_mix (C ABI in include/spectre_mix.h and
+include/dct_mix.h).
 
 Argument marshalling only: every step of the mix runs in the library's CUDA
-kernels.  The functions carry the C names; :class:`SpectreMix` wraps a handle
-for use with torch tensors.  Importing this module loads the library and
+kernels.  The functions carry the C names; :class:`SpectreMix` and
+:class:`DctMix` wrap a handle for use with torch tensors.  Importing this module loads the library and
 raises if it has not been built -- there is no fallback path.
 """
 from __future__ import annotations
@@ -56,6 +57,11 @@ SIGNATURES = {
     "spectre_mix_error_string": (ctypes.c_char_p, [_i]),
     "spectre_mix_workspace_bytes": (ctypes.c_size_t, [_vp]),
     "spectre_mix_plan_info": (_i, [_vp] + [ctypes.POINTER(_i)] * 5),
+    "dct_mix_create": (_i, [ctypes.POINTER(_vp), _i, _i, ctypes.c_float]),
+    "dct_mix_run": (_i, [_vp, ctypes.c_longlong] + [_vp] * 4 + [ctypes.c_float] + [_vp] * 4),
+    "dct_mix_run_debug": (_i, [_vp, ctypes.c_longlong] + [_vp] * 4 + [ctypes.c_float] + [_vp] * 5),
+    "dct_mix_run_host": (_i, [_vp, ctypes.c_longlong] + [_vp] * 4 + [ctypes.c_float] + [_vp] * 4),
+    "dct_mix_destroy": (_i, [_vp]),
 }
 
 
@@ -319,6 +325,125 @@ class SpectreMix:
         if self.handle is not None:
             h, self.handle = self.handle, None
             spectre_mix_destroy(h)
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---------------------------------------------------------------------------
+# per-token DCT mix with spectral-entropy routing (include/dct_mix.h)
+# ---------------------------------------------------------------------------
+def dct_mix_create_status(d: int, dtype: int, eps: float = 1e-5) -> Tuple[int, Optional[int]]:
+    h = _vp()
+    code = _lib.dct_mix_create(ctypes.byref(h), d, dtype, eps)
+    return code, h.value
+
+
+def dct_mix_create(d: int, dtype: int, eps: float = 1e-5) -> int:
+    code, h = dct_mix_create_status(d, dtype, eps)
+    _check(code, "dct_mix_create")
+    return h
+
+
+def dct_mix_run(h: int, T: int, x, w, gamma, beta, tau: float, y, H, route, stream=None) -> None:
+    _check(_lib.dct_mix_run(h, T, _ptr(x), _ptr(w), _ptr(gamma), _ptr(beta), tau, _ptr(y),
+                            _ptr(H), _ptr(route), _stream(stream)), "dct_mix_run")
+
+
+def dct_mix_run_debug(h: int, T: int, x, w, gamma, beta, tau: float, y, H, route, mix,
+                      stream=None) -> None:
+    _check(_lib.dct_mix_run_debug(h, T, _ptr(x), _ptr(w), _ptr(gamma), _ptr(beta), tau, _ptr(y),
+                                  _ptr(H), _ptr(route), _ptr(mix), _stream(stream)),
+           "dct_mix_run_debug")
+
+
+def dct_mix_run_host(h: int, T: int, x, w, gamma, beta, tau: float, y, H, route,
+                     stream=None) -> None:
+    _check(_lib.dct_mix_run_host(h, T, _ptr(x), _ptr(w), _ptr(gamma), _ptr(beta), tau, _ptr(y),
+                                 _ptr(H), _ptr(route), _stream(stream)), "dct_mix_run_host")
+
+
+def dct_mix_destroy(h: Optional[int]) -> None:
+    _check(_lib.dct_mix_destroy(h), "dct_mix_destroy")
+
+
+def check_dct_arguments(d, dtype_code, x, w, gamma, beta, y, H, route, mix=None) -> int:
+    """Sizes and types of one DCT-mix run's tensors; returns T (token rows).
+    x and y hold T * d values of the plan's type; w, gamma, beta d fp32
+    values; H T fp32 values; route T uint8 values; mix (optional) T * d fp32."""
+    import torch
+
+    if x.numel() % d:
+        raise ValueError(f"x must hold whole rows of d = {d} values")
+    T = x.numel() // d
+    tok_type = torch.float32 if dtype_code == SPECTRE_F32 else torch.bfloat16
+    for name, t in (("x", x), ("y", y)):
+        if t.numel() != T * d or t.dtype != tok_type:
+            raise ValueError(f"{name} must hold T * d = {T * d} values of {tok_type}")
+    for name, t in (("w", w), ("gamma", gamma), ("beta", beta)):
+        if t.numel() != d or t.dtype != torch.float32:
+            raise ValueError(f"{name} must hold d = {d} fp32 values")
+    if H.numel() != T or H.dtype != torch.float32:
+        raise ValueError(f"H must hold T = {T} fp32 values")
+    if route.numel() != T or route.dtype != torch.uint8:
+        raise ValueError(f"route must hold T = {T} uint8 values")
+    if mix is not None and (mix.numel() != T * d or mix.dtype != torch.float32):
+        raise ValueError(f"mix must hold T * d = {T * d} fp32 values")
+    return T
+
+
+class DctMix:
+    """A DCT-mix plan for token rows of length d (Chiaroscuro Attention
+    summary: the orthonormal Type-II DCT of each token, its normalised
+    spectral entropy H, the route H <= tau, and LayerNorm(x + iDCT(DCT(x) * w))).
+
+    ``mix(x, w, gamma, beta, tau)`` takes x [..., d] on the GPU and returns
+    (y, H, route) shaped [..., d], [...], [...]; pass ``mix_out=`` (fp32, the
+    shape of x) to also receive iDCT(DCT(x) * w).
+    """
+
+    def __init__(self, d: int, dtype: str = "bf16", eps: float = 1e-5):
+        self.d = d
+        self.dtype_code = SPECTRE_F32 if dtype in ("f32", "float32", "fp32") else SPECTRE_BF16
+        self.eps = eps
+        self.handle = dct_mix_create(d, self.dtype_code, eps)
+
+    def __call__(self, x, w, gamma, beta, tau: float, y=None, H=None, route=None, mix_out=None,
+                 stream=None):
+        import torch
+
+        lead = tuple(x.shape[:-1])
+        if y is None:
+            y = torch.empty_like(x)
+        if H is None:
+            H = torch.empty(lead, dtype=torch.float32, device=x.device)
+        if route is None:
+            route = torch.empty(lead, dtype=torch.uint8, device=x.device)
+        T = check_dct_arguments(self.d, self.dtype_code, x, w, gamma, beta, y, H, route, mix_out)
+        if mix_out is None:
+            dct_mix_run(self.handle, T, x, w, gamma, beta, tau, y, H, route, stream)
+        else:
+            dct_mix_run_debug(self.handle, T, x, w, gamma, beta, tau, y, H, route, mix_out, stream)
+        return y, H, route
+
+    def run_host(self, x, w, gamma, beta, tau: float, y, H, route, stream=None):
+        T = check_dct_arguments(self.d, self.dtype_code, x, w, gamma, beta, y, H, route)
+        dct_mix_run_host(self.handle, T, x, w, gamma, beta, tau, y, H, route, stream)
+        return y, H, route
+
+    def close(self) -> None:
+        if self.handle is not None:
+            h, self.handle = self.handle, None
+            dct_mix_destroy(h)
 
     def __enter__(self):
         return self

@@ -135,8 +135,10 @@ template <> struct Dft<16> {
     }
 };
 
-// exp(-2*pi*i*e/64), filled from the host at plan creation.  Defined here,
-// so exactly one translation unit (kernels.cu) includes this header.
+// exp(-2*pi*i*e/64), filled from the host at plan creation by kernels.cu.
+// Each translation unit that includes this header gets its own copy, and only
+// kernels.cu's is filled: other units (dct_mix.cu) use Dft<R> for R <= 16 only,
+// never Dft<32> or Dft<64>.
 static __constant__ float2 c_w64[64];
 
 // Composite R = R1 * R2 (R2 <= 16): length-R1 DFTs over samples r, r+R2, ...

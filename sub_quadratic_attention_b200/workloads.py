@@ -130,3 +130,83 @@ def make_inputs(w: Workload, seed_offset: int = 0) -> Dict[str, torch.Tensor]:
     else:
         out["beta"] = torch.randn(w.C, generator=g, dtype=torch.float32) * 0.1
     return out
+
+
+# ---------------------------------------------------------------------------
+# per-token DCT mix workloads
+# ---------------------------------------------------------------------------
+@dataclass(frozen=True)
+class DctWorkload:
+    """Token rows x[B, L, d] for the DCT mix.
+
+    Recipe (``make_dct_inputs``): a CPU generator seeded with ``2000 + index``;
+    draw order: the smooth/white choice per token, white rows, smooth-row
+    noise, w, gamma, beta.  Each token is, with probability 1/2, white
+    (N(0,1) i.i.d. over d) or smooth (a circular moving average of N(0,1)
+    noise over a window of d/16 along d, scaled back to unit variance), so
+    the spectral entropies spread over both sides of tau.  w ~ U(0,1),
+    gamma ~ N(1, 0.1), beta ~ N(0, 0.1); eps = 1e-5.  tau = 0.8954 at
+    d = 1024 (the threshold the page quotes for its 400M model, whose width
+    is 1024); the page gives none for d = 256, where 0.75 splits the smooth
+    rows (H about 0.5 to 0.6) from the white ones (about 0.87).
+    """
+    name: str
+    index: int
+    B: int
+    L: int
+    d: int
+    dtype: str
+    eps: float = 1e-5
+    tau: float = 0.8954
+
+    @property
+    def T(self) -> int:
+        return self.B * self.L
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    def algorithmic_bytes(self) -> int:
+        """x read, y written, H (fp32) and route (1 byte) written per token,
+        w, gamma, beta read once."""
+        return self.T * (2 * self.d * self.elem_bytes + 5) + 3 * self.d * 4
+
+
+DCT_WORKLOADS: Dict[str, DctWorkload] = {w.name: w for w in [
+    DctWorkload("dct_tiny_fp32", 0, B=1, L=37, d=64, dtype="f32", tau=0.75),
+    # the two model widths the page gives (d = 256 and 1024), sequence length 256
+    DctWorkload("dct_d256", 1, B=2048, L=256, d=256, dtype="bf16", tau=0.75),
+    DctWorkload("dct_d1024", 2, B=512, L=256, d=1024, dtype="bf16"),
+]}
+
+
+def dct_custom(B: int, L: int, d: int, dtype: str = "f32", index: int = 100,
+               tau: float = 0.8954) -> DctWorkload:
+    return DctWorkload("dct_custom", index, B=B, L=L, d=d, dtype=dtype, tau=tau)
+
+
+def make_dct_inputs(w: DctWorkload, seed_offset: int = 0) -> Dict[str, torch.Tensor]:
+    """Draw x [B, L, d], w, gamma, beta [d] on the CPU for workload ``w``
+    (``seed_offset`` gives each rank of a multi-GPU run its own tokens)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(2000 + w.index + seed_offset)
+    T, d = w.T, w.d
+    smooth = torch.rand(T, generator=g) < 0.5
+    x = torch.randn((T, d), generator=g, dtype=torch.float32)
+    ns = int(smooth.sum())
+    if ns:
+        win = max(1, d // 16)
+        e = torch.randn((ns, d), generator=g, dtype=torch.float32)
+        c = torch.cumsum(torch.cat([e, e[:, :win]], dim=1), dim=1)
+        avg = (c[:, win - 1:win - 1 + d] - torch.cat([torch.zeros(ns, 1), c[:, :d - 1]], dim=1))
+        x[smooth] = avg / math.sqrt(win)
+    out = {"x": x.reshape(w.B, w.L, d).to(w.torch_dtype)}
+    out["w"] = torch.rand(d, generator=g, dtype=torch.float32)
+    out["gamma"] = torch.randn(d, generator=g, dtype=torch.float32) * 0.1 + 1.0
+    out["beta"] = torch.randn(d, generator=g, dtype=torch.float32) * 0.1
+    return out

@@ -21,7 +21,7 @@ def _declared_functions():
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         for m in re.finditer(r"\b([a-z_][a-z0-9_]*)\s*\(", text):
             name = m.group(1)
-            if name.startswith("spectre_") and name not in names:
+            if name.startswith(("spectre_", "dct_mix_")) and name not in names:
                 names.append(name)
     return names
 
@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     names = _declared_functions()
     for required in ["spectre_mix_create", "spectre_mix_run", "spectre_mix_run_debug",
                      "spectre_mix_run_host", "spectre_mix_destroy", "spectre_mix_error_string",
-                     "spectre_mix_workspace_bytes", "spectre_mix_plan_info"]:
+                     "spectre_mix_workspace_bytes", "spectre_mix_plan_info", "dct_mix_create",
+                     "dct_mix_run", "dct_mix_run_debug", "dct_mix_run_host", "dct_mix_destroy"]:
         assert required in names
 
 
@@ -118,4 +119,36 @@ def test_create_without_a_device_reports_device_error():
     from sub_quadratic_attention_b200 import binding as b
 
     st, h = b.spectre_mix_create_status(1, 256, 1, 16, 129, 0)
+    assert st == b.SPECTRE_ERR_DEVICE and h is None
+
+
+@pytest.mark.parametrize("args,code", [
+    ((32, 0), "SPECTRE_ERR_UNSUPPORTED_L"),        # d below 64
+    ((96, 0), "SPECTRE_ERR_UNSUPPORTED_L"),        # not a power of two
+    ((2048, 1), "SPECTRE_ERR_UNSUPPORTED_L"),      # above 1024
+    ((256, 2), "SPECTRE_ERR_ARG"),                 # dtype
+])
+def test_dct_create_validates_before_touching_the_device(args, code):
+    from sub_quadratic_attention_b200 import binding as b
+
+    st, h = b.dct_mix_create_status(*args)
+    assert st == getattr(b, code) and h is None
+    for eps in (0.0, float("nan")):
+        st, h = b.dct_mix_create_status(256, 0, eps)
+        assert st == b.SPECTRE_ERR_ARG and h is None
+
+
+def test_dct_null_handle_paths():
+    from sub_quadratic_attention_b200 import binding as b
+
+    assert b._lib.dct_mix_destroy(None) == b.SPECTRE_OK
+    assert b._lib.dct_mix_run(None, 4, *([None] * 4), 0.5, *([None] * 4)) == b.SPECTRE_ERR_ARG
+    assert b._lib.dct_mix_run_host(None, 4, *([None] * 4), 0.5, *([None] * 4)) == b.SPECTRE_ERR_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_dct_create_without_a_device_reports_device_error():
+    from sub_quadratic_attention_b200 import binding as b
+
+    st, h = b.dct_mix_create_status(256, 1)
     assert st == b.SPECTRE_ERR_DEVICE and h is None

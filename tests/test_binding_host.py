@@ -59,3 +59,31 @@ def test_wrong_debug_output_is_rejected():
 def test_block_len_must_divide_L(block_len):
     with pytest.raises(ValueError):
         b.SpectreMix(1, 64, 1, 16, block_len=block_len)
+
+
+def _dct_args(T=5, d=64, dtype=torch.bfloat16):
+    return dict(x=torch.zeros(T, d, dtype=dtype), w=torch.ones(d), gamma=torch.ones(d),
+                beta=torch.zeros(d), y=torch.zeros(T, d, dtype=dtype),
+                H=torch.zeros(T), route=torch.zeros(T, dtype=torch.uint8))
+
+
+def test_dct_arguments_return_the_row_count():
+    a = _dct_args()
+    assert b.check_dct_arguments(64, b.SPECTRE_BF16, **a) == 5
+    a = _dct_args(T=0, dtype=torch.float32)
+    assert b.check_dct_arguments(64, b.SPECTRE_F32, **a, mix=torch.zeros(0, 64)) == 0
+
+
+@pytest.mark.parametrize("field,bad", [
+    ("x", torch.zeros(5, 63, dtype=torch.bfloat16)),
+    ("y", torch.zeros(5, 64, dtype=torch.float32)),
+    ("w", torch.ones(32)),
+    ("gamma", torch.ones(64, dtype=torch.float64)),
+    ("H", torch.zeros(4)),
+    ("route", torch.zeros(5, dtype=torch.bool)),
+])
+def test_dct_wrong_size_or_type_is_rejected(field, bad):
+    a = _dct_args()
+    a[field] = bad
+    with pytest.raises(ValueError):
+        b.check_dct_arguments(64, b.SPECTRE_BF16, **a)
