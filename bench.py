@@ -124,6 +124,28 @@ def ncu_traffic(workload: str, path: str = "spectre", kernels: int = 3):
     return None, {}
 
 
+def method_flops(w) -> float:
+    """The method's own arithmetic per step, counted on a radix-2 model: four
+    real transforms of length L per channel (q, k, v forward, out inverse) at
+    2.5 L log2 L flops each, about 14 flops per kept bin for the gated
+    product, and about 10 per element for the residual and LayerNorm."""
+    lg = math.log2(w.L)
+    return w.B * w.C * (4 * 2.5 * w.L * lg + 14 * w.F) + 10 * w.B * w.L * w.C
+
+
+def alu_roofline(flops: float, ms: float, sm_mhz) -> dict:
+    """The plain-ALU ceiling beside the HBM fraction: NUM_SMS x
+    FP32_LANES_PER_SM fp32 lanes, 2 flops a fused multiply-add, at the
+    median SM clock seen under load (the nominal 1965 MHz if none)."""
+    mhz = float(sm_mhz) if sm_mhz else 1965.0
+    peak = NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "alu", "method_flops": flops, "achieved": round(achieved, 3),
+            "peak": round(peak, 2), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_source": f"{NUM_SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 flops (FMA) at "
+                           f"{mhz:.0f} MHz"}
+
+
 def dominant_roofline(alg_bytes, units, kernel_ms, launches, kernel_traffic, names, peak_gbs):
     """Roofline of the dominant kernel (the largest time per step).
 
@@ -454,6 +476,7 @@ def native_arm(args, w, rank, world, local_rank):
                  "frac_of_8TBps_nominal": round(achieved / 8000.0, 4), "traffic": traffic,
                  "algorithmic_bytes": alg_bytes,
                  "scope": "whole step: algorithmic bytes over the timed step time"},
+        "alu": alu_roofline(method_flops(pw), ms_per_step, clocks.get("sm_mhz")),
         "kernels": kernels, "dominant_kernel": names[dom],
         "kernels_note": "per-kernel times from the profiled entry point, which runs the launches "
                         "one after another on one stream (sequential step "
@@ -507,6 +530,14 @@ def native_arm(args, w, rank, world, local_rank):
 # ---------------------------------------------------------------------------
 def dct_metric(w) -> str:
     return (f"dct-mix tokens/s at B{w.B} L{w.L} d{w.d} {w.dtype}; achieved HBM GB/s vs peak")
+
+
+def dct_method_flops(w) -> float:
+    """Per token: its half of one d-point complex FFT each way (5 d log2 d
+    flops per transform, shared by two rows), about 30 flops per coefficient
+    for the split, entropy, filter and re-twiddle, and about 10 per element
+    for the residual and LayerNorm."""
+    return w.T * (5.0 * w.d * math.log2(w.d) + 40.0 * w.d)
 
 
 def dct_config(w, world):
@@ -667,6 +698,7 @@ def dct_arm(args, w, rank, world, local_rank):
         "scope": "the step's one kernel: algorithmic bytes per token (x read and y written, "
                  "d values each, H and route written; w, gamma, beta once per launch) x the "
                  "tokens of a launch, over its CUDA-event time",
+        "alu": alu_roofline(dct_method_flops(w), ms_per_step, clocks.get("sm_mhz")),
     }
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

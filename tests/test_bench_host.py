@@ -89,3 +89,16 @@ def test_block_view_keeps_memory_and_scales_F():
 
     with pytest.raises(SystemExit):
         bench.block_view(w, inp, 100)
+
+
+def test_alu_ceiling_and_method_flops():
+    from sub_quadratic_attention_b200.workloads import DCT_WORKLOADS, WORKLOADS
+
+    f = bench.method_flops(WORKLOADS["bf16_long"])
+    assert abs(f / 1e9 - 5.76) < 0.02                 # about 5.8 GFLOP per step
+    r = bench.alu_roofline(f, 0.5, 1965)
+    assert abs(r["peak"] - 148 * 128 * 2 * 1.965e9 / 1e12) < 0.01
+    assert abs(r["achieved"] - f / 0.5e-3 / 1e12) < 1e-3 and r["bound"] == "alu"
+    assert bench.alu_roofline(f, 0.5, None)["peak"] == r["peak"]
+    w = DCT_WORKLOADS["dct_d1024"]
+    assert bench.dct_method_flops(w) == w.T * (5 * 1024 * 10 + 40 * 1024)
