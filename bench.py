@@ -339,7 +339,18 @@ def block_view(w, inputs, n):
 # ---------------------------------------------------------------------------
 # native arm
 # ---------------------------------------------------------------------------
-def native_arm(args, w, rank, world, local_rank):
+def _device(local_rank, device):
+    """The rank's CUDA device, made current; ``device`` overrides it (the CPU
+    tests of the JSON assembly run the arms with a fake library)."""
+    import torch
+
+    if device is not None:
+        return device
+    torch.cuda.set_device(local_rank)
+    return torch.device("cuda", local_rank)
+
+
+def native_arm(args, w, rank, world, local_rank, device=None):
     import torch
     import torch.distributed as dist
 
@@ -347,8 +358,7 @@ def native_arm(args, w, rank, world, local_rank):
     from sub_quadratic_attention_b200.ranks import job_throughput, max_over_ranks, rank_seed_offset
     from sub_quadratic_attention_b200.workloads import make_inputs
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+    dev = _device(local_rank, device)
     inputs = make_inputs(w, seed_offset=rank_seed_offset(rank))
     pw = w          # the shape the plan runs: w itself, or its blocks in blockwise mode
     if args.block_len:
@@ -600,7 +610,7 @@ def dct_reference_arm(args, w, rank, world):
     }), flush=True)
 
 
-def dct_arm(args, w, rank, world, local_rank):
+def dct_arm(args, w, rank, world, local_rank, device=None):
     import torch
     import torch.distributed as dist
 
@@ -608,8 +618,7 @@ def dct_arm(args, w, rank, world, local_rank):
     from sub_quadratic_attention_b200.ranks import job_throughput, max_over_ranks, rank_seed_offset
     from sub_quadratic_attention_b200.workloads import make_dct_inputs
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+    dev = _device(local_rank, device)
     inputs = make_dct_inputs(w, seed_offset=rank_seed_offset(rank))
     d = {k: v.to(dev) for k, v in inputs.items()}
     lead = (w.B, w.L)
