@@ -44,7 +44,7 @@ def _worker(rank, world, port, results):
 def test_two_gloo_ranks_share_only_the_timing():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of a multi-threaded test process
     results = mgr.dict()
     mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
     r0, r1 = results[0], results[1]
