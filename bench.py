@@ -124,6 +124,15 @@ def ncu_traffic(workload: str, path: str = "spectre", kernels: int = 3):
     return None, {}
 
 
+def path_dtype(w, slice_pass: str) -> str:
+    """What the path computes in: fp32 arithmetic on the CUDA cores, and for
+    the tensor-core slice pass fp16 DFT operands with fp32 accumulation."""
+    io = "bf16 I/O" if w.dtype == "bf16" else "f32 I/O"
+    if slice_pass == "tensor_cores":
+        return f"f32 ({io}; tensor-core DFT passes: f16 operands, f32 accumulate)"
+    return f"f32 ({io})"
+
+
 def method_flops(w) -> float:
     """The method's own arithmetic per step, counted on a radix-2 model: four
     real transforms of length L per channel (q, k, v forward, out inverse) at
@@ -520,8 +529,9 @@ def native_arm(args, w, rank, world, local_rank, device=None):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (seeded; shapes and distributions of the bf16 long workload)",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": path_dtype(w, mix.slice_pass),
+            "data": f"synthetic (seeded; shapes and distributions of the {w.name} workload)",
             "config": config_dict(w, world, pw),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -70,9 +70,9 @@ enum spectre_status {
 
 /*
  * Create a plan for one problem shape.  Validates the shape, picks the
- * decomposition L = R * M, computes the twiddle tables in double precision
- * on the host (stored as fp32) and allocates the workspace on the current
- * CUDA device.  Synchronous.
+ * decomposition L = R * M, allocates the twiddle tables and the workspace on
+ * the current CUDA device and fills the tables there (double-precision
+ * sines and cosines, stored as fp32).  Synchronous.
  *   out   : receives the handle (set to NULL on failure).
  *   B     : batch rows; L: sequence length; H: heads; D: channels per head.
  *   F     : number of low-frequency rfft bins kept (F = L/2 + 1 keeps all).
@@ -155,9 +155,11 @@ int spectre_mix_run_profiled(spectre_mix_t h, const void *q, const void *k,
  * over from the previous call.
  *
  *   Returns SPECTRE_ERR_SCRATCH when the tables plus the workspace of this
- *   shape (what spectre_mix_workspace_bytes reports for the same shape's
- *   plan, without staging) exceed the scratch; other errors as
- *   spectre_mix_create/spectre_mix_run.
+ *   shape (exactly what spectre_mix_workspace_bytes reports for the same
+ *   shape's plan before any spectre_mix_run_host call adds staging) exceed
+ *   the scratch; other errors as spectre_mix_create/spectre_mix_run.
+ *   No error word is kept for this path: if a bounded tensor-core wait
+ *   gives up, y comes out NaN (see spectre_mix_device_status).
  *
  * The first call on a device looks up the scratch's device address and loads
  * constant twiddles (synchronous); make that first call before any stream
@@ -192,7 +194,14 @@ enum spectre_option {
      * conj(G[L - f]), so the output stays real; the imaginary parts at DC
      * and Nyquist are dropped, as an inverse real FFT does.  The
      * no-allocation entry point takes real gates only. */
-    SPECTRE_OPT_COMPLEX_GATE = 3
+    SPECTRE_OPT_COMPLEX_GATE = 3,
+    /* 0 (default).  1: for tests of the failure path only.  In every
+     * tensor-core slice launch, block 0 issues no MMA and waits only a few
+     * 1 ms polls on its MMA barrier, so that wait gives up with nothing in
+     * flight: the run's y is NaN and spectre_mix_device_status reports
+     * SPECTRE_ERR_TIMEOUT.  No effect on plans that take the CUDA-core slice
+     * pass. */
+    SPECTRE_OPT_TEST_WAIT_TIMEOUT = 4
 };
 
 enum spectre_norm {
@@ -222,8 +231,12 @@ int spectre_mix_slice_pass(spectre_mix_t h);
 /*
  * Synchronise `stream` and report device-side failures of the handle's
  * earlier runs: SPECTRE_ERR_TIMEOUT if a bounded wait for a tensor-core MMA
- * gave up in any run since the last call (those runs' outputs are invalid),
- * else SPECTRE_OK.  Clears the recorded failure.
+ * gave up in any run since the last call, else SPECTRE_OK.  Clears the
+ * recorded failure.  A block whose wait gives up (after about 4 s) stops,
+ * releases its tensor memory and sets the scales of the slices it did not
+ * finish to NaN, so every y of that run is NaN: the failure is visible in
+ * the output as well (this is how spectre_mix_run_noalloc, which keeps no
+ * error word, reports it).
  */
 int spectre_mix_device_status(spectre_mix_t h, void *stream);
 

@@ -19,7 +19,7 @@
  *   m_n  = sum_k s_k (w_k X_k) cos(pi (2n+1) k / (2d))   (orthonormal inverse)
  *   y    = LayerNorm_d(x + m; gamma, beta, eps)
  *
- * Readings of points the pages leave open (each is listed in the design notes):
+ * Readings of points the pages leave open:
  *   - the DCT is orthonormal: the pages call it an orthogonal transform, and
  *     only then is the power spectrum the energy per basis vector;
  *   - the entropy is normalised by ln d so that it lies in [0, 1] as stated;

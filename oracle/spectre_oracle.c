@@ -18,7 +18,7 @@
  *     out[b,:,c] = irfft(O, n=L)
  *   y[b,t,:] = LayerNorm_C(out[b,t,:] + x[b,t,:]; gamma, beta, eps)
  *
- * Readings of points the pages leave open (each is listed in the design notes):
+ * Readings of points the pages leave open:
  *   - forward transform unscaled, inverse scaled by 1/L (the default norm of
  *     the fft/ifft calls in the §2.2 pseudocode);
  *   - real-input transforms (rfft/irfft): for real q,k,v and a real gate they

@@ -30,6 +30,7 @@ SPECTRE_ERR_TIMEOUT = -8
 SPECTRE_OPT_TENSOR_CORES = 1
 SPECTRE_OPT_NORM = 2
 SPECTRE_OPT_COMPLEX_GATE = 3
+SPECTRE_OPT_TEST_WAIT_TIMEOUT = 4
 
 # enum spectre_norm, keyed as in the oracle
 SPECTRE_NORM = {"post_ln": 0, "pre_ln": 1, "post_rms": 2, "pre_rms": 3}

@@ -21,16 +21,18 @@ struct PathGeom {
     int B, L, H, D, C, F, dtype;
     float eps;
     int R, M, NF;
-    int W;               // channels per wave (A of one wave kept in L2)
+    int a16;             // A stored as bf16 (re, im) pairs (bf16 I/O, slice pass does not park in A)
+    int regions;         // A regions: 1 (chunks run one after another and reuse it) or 2 (alternating streams)
     int p16;             // P stored as fp16 with per-slice scales (bf16 I/O)
     int T2C, ZS;         // inverse row pass
     int inv_reg;         // register-resident LayerNorm variant
     int tc_mode;         // option: slice pass on the tensor cores where mma_ok (1) or CUDA cores (0)
     int norm_mode;       // option: enum spectre_norm
     int cgate;           // option: complex gate
+    int test_stall;      // option: the wait-timeout test (tensor-core slice pass)
     int mma_ok;          // the DFT-64 MMA slice pass applies (M = 4096, fp16 P, few live groups)
     int nsm;             // multiprocessors of the device
-    int chunk;           // channels per pipeline chunk (multiple of 64, or C)
+    int chunk;           // channels per chunk (a multiple of 64, or C)
     size_t a_bytes, p_bytes, s_bytes;
 };
 
@@ -40,7 +42,7 @@ struct PathBuffers {
     SliceTables tabs;
     const float2 *twMM;  // M = 4096: w_4096^{n2 k1} as [k1][n2]
     const void *w64op;   // M = 4096: the fp16 DFT-64 operand
-    float2 *A;           // [3][B][W][NF][M]
+    void *A;             // regions x [3][B][chunk][NF][M], float2 or bf16 pairs (a16)
     void *P;             // [B][C][NF][M] float2 or __half2
     float *pscale;       // [B][C][NF]
     int *err;            // device error word (bit 0: a tensor-core wait timed out)
@@ -79,6 +81,18 @@ bool fault_requested(const char *what) {
 }
 
 bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// Fraction of L2 that one chunk's A (or both regions' A) may fill.  Measured
+// on B200: data written by one kernel is read back by the next entirely from
+// L2 up to about 64 MB (of 126 MB); at 96 MB about 40 MB comes from DRAM.
+#ifndef SPECTRE_L2_FRACTION
+#define SPECTRE_L2_FRACTION 0.45
+#endif
+#ifndef SPECTRE_A_REGIONS
+#define SPECTRE_A_REGIONS 1
+#endif
+constexpr double kL2Fraction = SPECTRE_L2_FRACTION;
+constexpr int kARegions = SPECTRE_A_REGIONS;
 
 // L = R * M: R-point row transforms, M-point slice transforms.
 bool choose_split(int L, int *R, int *M) {
@@ -135,8 +149,10 @@ void free_handle(spectre_mix_s *h) {
 }
 
 // Validate a shape and derive its geometry.  l2_bytes sizes the channel
-// waves: one wave's A (3 signals x B x W channels x (R/2+1) x M complex fp32)
-// is kept within half of L2 so the slice pass reads it back from L2.
+// chunks: one chunk's A (3 signals x B x chunk channels x (R/2+1) x M complex
+// values) is kept within a fraction of L2, so the slice pass reads A back
+// from L2 and the next chunk's row pass overwrites those lines in L2 rather
+// than DRAM receiving them.
 int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2_bytes, PathGeom *g) {
     if (B < 1 || B > 65535 || H < 1 || D < 1 || L < 1) return SPECTRE_ERR_ARG;
     if (dtype != SPECTRE_F32 && dtype != SPECTRE_BF16) return SPECTRE_ERR_ARG;
@@ -154,21 +170,9 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     g->R = R; g->M = M; g->NF = NF;
     g->ZS = ZS;
     g->p16 = dtype == SPECTRE_BF16 ? 1 : 0;
-    // channel waves: with kWaveL2Fraction > 0, one wave's A is sized to that
-    // fraction of L2 so the slice pass could read it back from L2.  Measured on
-    // B200 for the bf16 long workload, waves were slower (each wave's grid
-    // fills the SMs only ~1.2 times and L2 still wrote most of A back to
-    // DRAM), so the plan uses a single wave.
-    constexpr double kWaveL2Fraction = 0.0;
-    const size_t per_ch = (size_t)3 * B * NF * M * sizeof(float2);
-    const size_t budget = (size_t)(kWaveL2Fraction * (double)l2_bytes);
-    int W = C;
-    if (budget > 0 && per_ch * (size_t)C > budget) {
-        size_t w = budget / per_ch;
-        w -= w % 64;
-        if (w >= 64) W = (int)w;
-    }
-    g->W = W;
+    // A in bf16 pairs where the slice pass reads it (it parks its running
+    // product in fp32 A only for the longest slices)
+    g->a16 = (g->p16 && !slice_parks_in_A(M)) ? 1 : 0;
     // inverse row pass: register-resident LayerNorm when a block of
     // T2C x ceil(C/2) <= 1024 threads covers the channels; else the
     // shared-memory variant (R rows x T2C x padded C floats per block)
@@ -186,7 +190,7 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     // tensor-core slice pass: M = 4096 as two DFT-64 MMA passes, for fp16 P,
     // when no slice has more than kMmaMaxGroups live k2 groups
     g->mma_ok = 0;
-    if (M == 4096 && g->p16) {
+    if (M == 4096 && g->p16 && g->a16) {
         int worst = 0;
         for (int f1 = 0; f1 < NF; f1++) {
             int n = 0;
@@ -198,12 +202,24 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     g->tc_mode = 1;
     g->norm_mode = SPECTRE_NORM_POST_LN;
     g->cgate = 0;
+    g->test_stall = 0;
     g->nsm = 148;
-    // pipeline chunks: four channel chunks when each still fills the GPU
-    g->chunk = C;
-    if (W == C && C >= 256) g->chunk = (int)align_up((size_t)(C + 3) / 4, 64);
+    // channel chunks: the largest multiple of 64 channels whose A fits the L2
+    // budget (at least 64), all of C when that fits
+    const size_t per_ch = (size_t)3 * B * NF * M * (g->a16 ? 4 : 8);
+    const int regions = kARegions;
+    const size_t budget = (size_t)(kL2Fraction * (double)l2_bytes) / (size_t)regions;
+    int chunk = C;
+    if (per_ch * (size_t)C > budget && C > 64) {
+        size_t w = budget / per_ch;
+        w -= w % 64;
+        chunk = (int)(w < 64 ? 64 : w);
+        if (chunk > C) chunk = C;
+    }
+    g->chunk = chunk;
+    g->regions = chunk < C ? regions : 1;
     const size_t slices = (size_t)B * C * NF;
-    g->a_bytes = align_up((size_t)3 * B * W * NF * M * sizeof(float2), 256);
+    g->a_bytes = align_up((size_t)g->regions * per_ch * (size_t)chunk, 256);
     // fp16 P interleaves channel pairs: 2 ceil(C / 2) channel lanes
     const size_t pslices = g->p16 ? (size_t)B * 2 * ((C + 1) / 2) * NF : slices;
     g->p_bytes = align_up(pslices * M * (g->p16 ? 4 : 8), 256);
@@ -211,27 +227,86 @@ int make_geom(int B, int L, int H, int D, int F, int dtype, float eps, size_t l2
     return SPECTRE_OK;
 }
 
+// Layout of the plan's twiddle tables in one device buffer, as segments the
+// table kernel fills (fp64 sincospi, stored fp32): the L-point table w_L^e
+// (e <= L/2), the slice-pass tables of each pass and direction, and for
+// M = 4096 the twiddles w_4096^{n2 k1} ([k1][n2]) and the fp16 DFT-64 operand.
+// The handle and the no-allocation entry point use this one layout and the
+// one kernel, so both compute bit-identical tables.
+struct TableLayout {
+    TableSegs segs;
+    size_t bytes;        // rounded up to 256
+    long long off_slice[2][kMaxPasses];
+    long long off_mm, off_op;   // -1 when absent
+};
+
+TableLayout table_layout(const PathGeom &g) {
+    TableLayout t;
+    t.segs.n = 0;
+    t.off_mm = t.off_op = -1;
+    for (int d = 0; d < 2; d++)
+        for (int p = 0; p < kMaxPasses; p++) t.off_slice[d][p] = -1;
+    const RadList sch = make_schedule(g.M);
+    size_t n = (size_t)g.L / 2 + 1;
+    t.segs.seg[t.segs.n++] = TableSeg{0, (long long)n, 0, (long long)g.L};
+    for (int d = 0; d < 2; d++) {
+        int ns = 1;
+        for (int p = 0; p < sch.n; p++) {
+            const int r = d == 0 ? sch.r[p] : sch.r[sch.n - 1 - p];
+            if (p > 0) {
+                const size_t base = align_up(n, 2);
+                t.off_slice[d][p] = (long long)base;
+                t.segs.seg[t.segs.n++] = TableSeg{(long long)base, (long long)ns * r, (long long)ns,
+                                                  (long long)ns * r};
+                n = base + (size_t)ns * r;
+            }
+            ns *= r;
+        }
+    }
+    if (g.M == 4096) {
+        size_t base = align_up(n, 2);
+        t.off_mm = (long long)base;
+        t.segs.seg[t.segs.n++] = TableSeg{(long long)base, 4096, 64, 4096};
+        base = align_up(base + 4096, 2);
+        t.off_op = (long long)base;
+        t.segs.seg[t.segs.n++] = TableSeg{(long long)base, 4096, -1, 64};
+        n = base + 4096;
+    }
+    t.bytes = align_up(n * sizeof(float2), 256);
+    return t;
+}
+
+// Table pointers of a plan whose tables start at tw.
+void bind_tables(const TableLayout &t, float2 *tw, PathBuffers *bf) {
+    bf->twL = tw;
+    for (int d = 0; d < 2; d++)
+        for (int p = 0; p < kMaxPasses; p++)
+            bf->tabs.tw[d][p] = t.off_slice[d][p] >= 0 ? tw + t.off_slice[d][p] : nullptr;
+    bf->twMM = t.off_mm >= 0 ? tw + t.off_mm : nullptr;
+    bf->w64op = t.off_op >= 0 ? static_cast<const void *>(tw + t.off_op) : nullptr;
+}
+
+// exp(-2 pi i e / 64), e < 64, for the constant bank of the R = 64 kernels
+void host_w64(float2 (&w64)[64]) {
+    for (int e = 0; e < 64; e++) {
+        double ang = -2.0 * M_PI * e / 64.0;
+        w64[e] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+}
+
 // Whether the slice pass runs on the tensor cores (option on and the plan in
 // the tensor-core kernel's range).
 bool uses_mma(const PathGeom &g) { return g.tc_mode == 1 && g.mma_ok; }
 
-// Channels per pipeline chunk.  Measured on B200 for the bf16 long workload:
-// four chunks suit the CUDA-core slice pass (0.573 ms per mix against 0.60 ms
-// unchunked); the tensor-core slice pass, whose blocks each carry a long
-// chain of dependent phases, does best with two (0.454 ms against 0.460 with
-// four and 0.464 unchunked), which keep more blocks per launch.
-int chunk_channels(const PathGeom &g) {
-    if (!uses_mma(g) || g.chunk >= g.W) return g.chunk;
-    return (int)align_up((size_t)(g.C + 1) / 2, 64);
-}
-
-// The launch sequence of one mix.  Per channel chunk (within each wave) the
-// row pass then the slice pass, then the inverse row pass with residual +
-// LayerNorm.  Each chunk has its own region of A, so with an auxiliary stream
-// the chunks alternate between `s` and `aux` and the row pass of chunk k + 1
-// runs while the slice pass of chunk k does; `aux` forks from and joins back
-// into `s`.  events (nullable, one per launch + 1) are recorded before every
-// launch and after the last; with events the schedule is single-stream.
+// The launch sequence of one mix: per channel chunk the row pass then the
+// slice pass, then the inverse row pass with residual + LayerNorm.  With one
+// A region the chunks run one after another on `s` and each overwrites the
+// previous chunk's A (still in L2).  With two regions the chunks alternate
+// between `s` and `aux` (and between the regions), so the row pass of chunk
+// k + 1 can run while the slice pass of chunk k does; `aux` forks from and
+// joins back into `s`.  events (nullable, one per launch + 1) are recorded
+// before every launch and after the last; with events the schedule is
+// single-stream.
 int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const void *k, const void *v,
                 const void *x, const float *G, const float *gamma, const float *beta, void *y,
                 float *out_f32, void *const *events, cudaStream_t s, cudaStream_t aux,
@@ -240,8 +315,10 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     auto mark = [&](cudaStream_t st) -> cudaError_t {
         return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), st) : cudaSuccess;
     };
-    const int chunk = chunk_channels(g);
-    const bool two = aux && !events && chunk < g.W;
+    const int chunk = g.chunk;
+    const bool two = aux && !events && g.regions == 2;
+    const size_t region_elems = (size_t)3 * g.B * chunk * g.NF * g.M;
+    const size_t elem = g.a16 ? 4 : 8;
     cudaError_t e = cudaSuccess;
     if (two) {
         e = cudaEventRecord(ev_fork, s);
@@ -249,43 +326,43 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
         if (e != cudaSuccess) return cuda_status(e);
     }
     int idx = 0;
-    for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
-        const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
-        for (int c_lo = w_lo; c_lo < w_hi; c_lo += chunk, idx++) {
-            const int Cw = w_hi - c_lo < chunk ? w_hi - c_lo : chunk;
-            cudaStream_t st = (two && (idx & 1)) ? aux : s;
-            // this chunk's region of A: [3][B][Cw][NF][M] at its offset in the wave
-            float2 *A = bf.A + (size_t)3 * g.B * (c_lo - w_lo) * g.NF * g.M;
-            RowsFwdArgs fa;
-            fa.q = q; fa.k = k; fa.v = v;
-            fa.A = A;
-            fa.twL = bf.twL;
-            fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
-            fa.c_lo = c_lo; fa.Cw = Cw;
-            fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
-            fa.nsm = g.nsm;
-            e = mark(st);
-            if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, st);
-            if (e != cudaSuccess) return cuda_status(e);
+    for (int c_lo = 0; c_lo < g.C; c_lo += chunk, idx++) {
+        const int Cw = g.C - c_lo < chunk ? g.C - c_lo : chunk;
+        cudaStream_t st = (two && (idx & 1)) ? aux : s;
+        // this chunk's region of A: [3][B][Cw][NF][M]
+        void *A = static_cast<char *>(bf.A) + (size_t)(idx % g.regions) * region_elems * elem;
+        RowsFwdArgs fa;
+        fa.q = q; fa.k = k; fa.v = v;
+        fa.A = A;
+        fa.a16 = g.a16;
+        fa.twL = bf.twL;
+        fa.B = g.B; fa.L = g.L; fa.M = g.M; fa.C = g.C;
+        fa.c_lo = c_lo; fa.Cw = Cw;
+        fa.vec2 = (g.C % 2 == 0) ? 1 : 0;
+        fa.nsm = g.nsm;
+        e = mark(st);
+        if (e == cudaSuccess) e = launch_rows_fwd(g.R, g.dtype, fa, st);
+        if (e != cudaSuccess) return cuda_status(e);
 
-            SliceArgs sa;
-            sa.A = A; sa.P = bf.P; sa.pscale = bf.pscale; sa.twL = bf.twL; sa.G = G; sa.tabs = bf.tabs;
-            sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
-            sa.c_lo = c_lo; sa.Cw = Cw;
-            sa.p16 = g.p16;
-            sa.use_mma = uses_mma(g) ? 1 : 0;
-            sa.nsm = g.nsm;
-            sa.twMM = bf.twMM;
-            sa.w64op = bf.w64op;
-            sa.err = bf.err;
-            sa.nbins = g.L / 2 + 1;
-            sa.cgate = g.cgate;
-            sa.nslices = (long long)g.B * Cw * g.NF;
-            sa.invL = 1.0f / (float)g.L;
-            e = mark(st);
-            if (e == cudaSuccess) e = launch_slices(sa, st);
-            if (e != cudaSuccess) return cuda_status(e);
-        }
+        SliceArgs sa;
+        sa.A = A; sa.a16 = g.a16;
+        sa.P = bf.P; sa.pscale = bf.pscale; sa.twL = bf.twL; sa.G = G; sa.tabs = bf.tabs;
+        sa.B = g.B; sa.L = g.L; sa.R = g.R; sa.M = g.M; sa.C = g.C; sa.D = g.D; sa.F = g.F;
+        sa.c_lo = c_lo; sa.Cw = Cw;
+        sa.p16 = g.p16;
+        sa.use_mma = uses_mma(g) ? 1 : 0;
+        sa.nsm = g.nsm;
+        sa.twMM = bf.twMM;
+        sa.w64op = bf.w64op;
+        sa.err = bf.err;
+        sa.nbins = g.L / 2 + 1;
+        sa.cgate = g.cgate;
+        sa.test_stall = g.test_stall;
+        sa.nslices = (long long)g.B * Cw * g.NF;
+        sa.invL = 1.0f / (float)g.L;
+        e = mark(st);
+        if (e == cudaSuccess) e = launch_slices(sa, st);
+        if (e != cudaSuccess) return cuda_status(e);
     }
     if (two) {
         e = cudaEventRecord(ev_join, aux);
@@ -308,14 +385,7 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
     return SPECTRE_OK;
 }
 
-int launch_count(const PathGeom &g) {
-    int n = 0;
-    for (int w_lo = 0; w_lo < g.C; w_lo += g.W) {
-        const int w_hi = g.C - w_lo < g.W ? g.C : w_lo + g.W;
-        n += 2 * ((w_hi - w_lo + chunk_channels(g) - 1) / chunk_channels(g));
-    }
-    return n + 1;
-}
+int launch_count(const PathGeom &g) { return 2 * ((g.C + g.chunk - 1) / g.chunk) + 1; }
 
 size_t l2_size(int dev) {
     int v = 0;
@@ -340,7 +410,7 @@ const char *spectre_mix_error_string(int code) {
     case SPECTRE_ERR_NOMEM: return "out of memory";
     case SPECTRE_ERR_DEVICE: return "no usable sm_100 device, or the handle's device is not current";
     case SPECTRE_ERR_SCRATCH: return "problem needs more than the 64 MiB no-allocation scratch holds";
-    case SPECTRE_ERR_TIMEOUT: return "a bounded wait on the tensor cores timed out; results of the run are invalid";
+    case SPECTRE_ERR_TIMEOUT: return "a bounded wait on the tensor cores timed out; results of the run are invalid (y is NaN)";
     default: return "unknown status";
     }
 }
@@ -349,7 +419,7 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     if (!out) return SPECTRE_ERR_ARG;
     *out = nullptr;
     PathGeom g;
-    // validate with a provisional L2 size; the waves are re-derived below
+    // validate with a provisional L2 size; the chunks are re-derived below
     int st = make_geom(B, L, H, D, F, dtype, eps, (size_t)32 << 20, &g);
     if (st != SPECTRE_OK) return st;
     if (fault_requested("alloc")) return SPECTRE_ERR_NOMEM;
@@ -363,92 +433,31 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     if (!h) return SPECTRE_ERR_NOMEM;
     h->device = dev;
     h->g = g;
-    const int M = g.M;
 
-    // ---- twiddle tables (double on the host, stored fp32)
-    const RadList sch = make_schedule(M);
-    std::vector<float2> host;
-    const size_t nL = (size_t)L / 2 + 1;
-    host.resize(nL);
-    for (size_t e = 0; e < nL; e++) {
-        double ang = -2.0 * M_PI * (double)e / (double)L;
-        host[e] = make_float2((float)std::cos(ang), (float)std::sin(ang));
-    }
-    size_t offs[2][kMaxPasses] = {};
-    for (int d = 0; d < 2; d++) {
-        int ns = 1;
-        for (int p = 0; p < sch.n; p++) {
-            int r = d == 0 ? sch.r[p] : sch.r[sch.n - 1 - p];
-            if (p > 0) {
-                size_t base = align_up(host.size(), 2);
-                host.resize(base);
-                offs[d][p] = base;
-                for (int rr = 0; rr < r; rr++)
-                    for (int kk = 0; kk < ns; kk++) {
-                        long long e = (long long)kk * rr;
-                        double ang = -2.0 * M_PI * (double)e / (double)(ns * r);
-                        host.push_back(make_float2((float)std::cos(ang), (float)std::sin(ang)));
-                    }
-            }
-            ns *= r;
-        }
-    }
-    // M = 4096: the twiddles between the two DFT-64 passes and the fp16
-    // DFT-64 operand of the tensor-core slice pass
-    size_t off_mm = 0, off_op = 0;
-    if (M == 4096) {
-        off_mm = align_up(host.size(), 2);
-        host.resize(off_mm);
-        for (int k1 = 0; k1 < 64; k1++)
-            for (int n2 = 0; n2 < 64; n2++) {
-                double ang = -2.0 * M_PI * (double)(n2 * k1) / 4096.0;
-                host.push_back(make_float2((float)std::cos(ang), (float)std::sin(ang)));
-            }
-        off_op = align_up(host.size(), 2);
-        host.resize(off_op + 4096);
-        unsigned char *bytes = reinterpret_cast<unsigned char *>(host.data() + off_op);
-        for (int n = 0; n < 128; n++)
-            for (int kk = 0; kk < 128; kk++) {
-                long long ee;
-                int part;
-                dft64_operand_angle(n, kk, &ee, &part);
-                const double ang = -2.0 * M_PI * (double)ee / 64.0;
-                const double val = (part == 0 || part == 3) ? std::cos(ang)
-                                 : (part == 1 ? -std::sin(ang) : std::sin(ang));
-                const __half hv = __float2half_rn((float)(val / 64.0));
-                std::memcpy(bytes + dft64_operand_offset(n, kk), &hv, sizeof(hv));
-            }
-    }
+    // ---- twiddle tables: fp64 on the device (the table kernel), stored fp32
+    const TableLayout tl = table_layout(g);
     float2 w64[64];
-    for (int e = 0; e < 64; e++) {
-        double ang = -2.0 * M_PI * e / 64.0;
-        w64[e] = make_float2((float)std::cos(ang), (float)std::sin(ang));
-    }
-
+    host_w64(w64);
     cudaError_t e;
-    h->table_bytes = host.size() * sizeof(float2);
+    h->table_bytes = tl.bytes;
     e = cudaMalloc(&h->tables, h->table_bytes);
-    if (e == cudaSuccess) e = cudaMemcpy(h->tables, host.data(), h->table_bytes, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = launch_make_tables(static_cast<float2 *>(h->tables), tl.segs, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
     if (e == cudaSuccess) e = upload_w64(w64);
     if (e != cudaSuccess) {
         cudaGetLastError();
         free_handle(h);
         return cuda_status(e);
     }
-    h->bufs.twL = static_cast<float2 *>(h->tables);
-    h->bufs.twMM = M == 4096 ? h->bufs.twL + off_mm : nullptr;
-    h->bufs.w64op = M == 4096 ? static_cast<const void *>(h->bufs.twL + off_op) : nullptr;
+    bind_tables(tl, static_cast<float2 *>(h->tables), &h->bufs);
     {
         int nsm = 0;
         if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
             h->g.nsm = nsm;
         cudaGetLastError();
     }
-    for (int d = 0; d < 2; d++)
-        for (int p = 0; p < kMaxPasses; p++)
-            h->bufs.tabs.tw[d][p] = (p > 0 && p < sch.n) ? h->bufs.twL + offs[d][p] : nullptr;
 
-    // ---- workspace: A of one wave, P, P scales
+    // ---- workspace: A (one or two chunk regions), P, P scales
     h->ws_bytes = g.a_bytes + g.p_bytes + g.s_bytes;
     e = cudaMalloc(&h->ws, h->ws_bytes);
     if (e != cudaSuccess) {
@@ -457,12 +466,12 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
         return cuda_status(e);
     }
     char *base = static_cast<char *>(h->ws);
-    h->bufs.A = reinterpret_cast<float2 *>(base);
+    h->bufs.A = base;
     h->bufs.P = base + g.a_bytes;
     h->bufs.pscale = reinterpret_cast<float *>(base + g.a_bytes + g.p_bytes);
     h->bufs.err = reinterpret_cast<int *>(base + g.a_bytes + g.p_bytes + g.s_bytes - 256);
     e = cudaMemset(h->bufs.err, 0, sizeof(int));
-    if (e == cudaSuccess && g.chunk < g.W) {
+    if (e == cudaSuccess && g.regions == 2) {
         e = cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
@@ -589,38 +598,10 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     if (st != SPECTRE_OK) return st;
     make_geom(B, L, H, D, F, dtype, eps, l2_size(dev), &g);
 
-    // scratch layout: twiddle tables (as spectre_mix_create lays them out),
-    // then A of one wave, P and the P scales
-    const RadList sch = make_schedule(g.M);
-    TableSegs segs;
-    segs.n = 0;
-    size_t n_tab = (size_t)L / 2 + 1;
-    segs.seg[segs.n++] = TableSeg{0, (long long)n_tab, 0, (long long)L};
-    for (int d = 0; d < 2; d++) {
-        int ns = 1;
-        for (int p = 0; p < sch.n; p++) {
-            int r = d == 0 ? sch.r[p] : sch.r[sch.n - 1 - p];
-            if (p > 0) {
-                size_t base = align_up(n_tab, 2);
-                segs.seg[segs.n++] = TableSeg{(long long)base, (long long)ns * r, (long long)ns,
-                                              (long long)ns * r};
-                n_tab = base + (size_t)ns * r;
-            }
-            ns *= r;
-        }
-    }
-    long long seg_mm = -1, seg_op = -1;
-    if (g.M == 4096) {
-        size_t base = align_up(n_tab, 2);
-        seg_mm = segs.n;
-        segs.seg[segs.n++] = TableSeg{(long long)base, 4096, 64, 4096};
-        base = align_up(base + 4096, 2);
-        seg_op = segs.n;
-        segs.seg[segs.n++] = TableSeg{(long long)base, 4096, -1, 64};
-        n_tab = base + 4096;
-    }
-    const size_t tab_bytes = align_up(n_tab * sizeof(float2), 256);
-    const size_t need = tab_bytes + g.a_bytes + g.p_bytes + g.s_bytes;
+    // scratch layout: twiddle tables (the layout spectre_mix_create uses),
+    // then A, P and the P scales
+    const TableLayout tl = table_layout(g);
+    const size_t need = tl.bytes + g.a_bytes + g.p_bytes + g.s_bytes;
     if (need > kNoAllocScratchBytes) return SPECTRE_ERR_SCRATCH;
     if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
     void *scratch = nullptr;
@@ -633,26 +614,18 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     char *base = static_cast<char *>(scratch);
     PathBuffers bf;
     float2 *tw = reinterpret_cast<float2 *>(base);
-    bf.twL = tw;
-    bf.A = reinterpret_cast<float2 *>(base + tab_bytes);
-    bf.P = base + tab_bytes + g.a_bytes;
-    bf.pscale = reinterpret_cast<float *>(base + tab_bytes + g.a_bytes + g.p_bytes);
-    bf.err = nullptr;   // no error word: the no-allocation path reports launch errors only
-    bf.twMM = seg_mm >= 0 ? tw + segs.seg[seg_mm].offset : nullptr;
-    bf.w64op = seg_op >= 0 ? static_cast<const void *>(tw + segs.seg[seg_op].offset) : nullptr;
+    bind_tables(tl, tw, &bf);
+    bf.A = base + tl.bytes;
+    bf.P = base + tl.bytes + g.a_bytes;
+    bf.pscale = reinterpret_cast<float *>(base + tl.bytes + g.a_bytes + g.p_bytes);
+    bf.err = nullptr;   // no error word: a tensor-core wait that gives up poisons y with NaN
     {
         int nsm = 0;
         if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && nsm > 0)
             g.nsm = nsm;
         cudaGetLastError();
     }
-    {
-        int si = 1;
-        for (int d = 0; d < 2; d++)
-            for (int p = 0; p < kMaxPasses; p++)
-                bf.tabs.tw[d][p] = (p > 0 && p < sch.n) ? tw + segs.seg[si++].offset : nullptr;
-    }
-    e = launch_make_tables(tw, segs, s);
+    e = launch_make_tables(tw, tl.segs, s);
     if (e != cudaSuccess) return cuda_status(e);
     // single stream: this path creates no streams or events
     return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s, nullptr, nullptr,
@@ -673,6 +646,10 @@ int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     case SPECTRE_OPT_NORM:
         if (value < SPECTRE_NORM_POST_LN || value > SPECTRE_NORM_PRE_RMS) return SPECTRE_ERR_ARG;
         h->g.norm_mode = value;
+        return SPECTRE_OK;
+    case SPECTRE_OPT_TEST_WAIT_TIMEOUT:
+        if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
+        h->g.test_stall = value;
         return SPECTRE_OK;
     default: return SPECTRE_ERR_ARG;
     }
@@ -729,7 +706,7 @@ int spectre_mix_plan_info(spectre_mix_t h, int *R, int *M, int *slices_per_chann
     if (R) *R = h->g.R;
     if (M) *M = h->g.M;
     if (slices_per_channel) *slices_per_channel = h->g.NF;
-    if (channels_per_wave) *channels_per_wave = h->g.W;
+    if (channels_per_wave) *channels_per_wave = h->g.chunk;
     if (launches) *launches = launch_count(h->g);
     return SPECTRE_OK;
 }

@@ -20,6 +20,10 @@
 #include "fft_regs.cuh"
 #include "kernels.cuh"
 
+#ifndef SPECTRE_L2_HINTS
+#define SPECTRE_L2_HINTS 1
+#endif
+
 namespace spectre {
 
 // ---------------------------------------------------------------------------
@@ -55,6 +59,25 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// One complex value of A: fp32 (float2), or with A16 a bf16 (re, im) pair.
+// bf16 halves the intermediate's bytes; its 8-bit significand adds a
+// relative error of at most 2^-9 per value, well inside the bf16-input bar.
+template <bool A16> struct AElem;
+template <> struct AElem<false> {
+    using T = float2;
+    __device__ __forceinline__ static void store(float2 *p, float2 v) { *p = v; }
+    __device__ __forceinline__ static float2 load(const float2 *p) { return __ldg(p); }
+};
+template <> struct AElem<true> {
+    using T = __nv_bfloat162;
+    __device__ __forceinline__ static void store(__nv_bfloat162 *p, float2 v) {
+        *p = __floats2bfloat162_rn(v.x, v.y);
+    }
+    __device__ __forceinline__ static float2 load(const __nv_bfloat162 *p) {
+        return __bfloat1622float2(__ldg(p));
+    }
+};
+
 // ---------------------------------------------------------------------------
 // row pass: A[sig][b][c][f1][t2] = w_L^{f1 t2} sum_{t1} w_R^{f1 t1} sig[b][t1 M + t2][c]
 // Block: 256 threads = 8 warps over 8 t2 values x 32 channel pairs; a warp
@@ -64,9 +87,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 // (8 channel pairs) and its stores are 32-byte segments (4 consecutive t2) of
 // A, straight from registers.
 // ---------------------------------------------------------------------------
-template <int R, typename T>
+template <int R, typename T, bool A16>
 __global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwdArgs a) {
     constexpr int NF = R / 2 + 1;
+    using AT = typename AElem<A16>::T;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t2 = blockIdx.x * 8 + (warp & 1) * 4 + (lane & 3);
     const int cp = blockIdx.y * 32 + (warp >> 1) * 8 + (lane >> 2);
@@ -78,8 +102,8 @@ __global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwd
     const bool has1 = live && (c0 + 1 < cend);
     const size_t rowstride = (size_t)a.M * a.C;
     const size_t plane = (size_t)a.B * a.Cw * NF * a.M;
-    float2 *dst0 = a.A + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
-    float2 *dst1 = dst0 + (size_t)NF * a.M;
+    AT *dst0 = static_cast<AT *>(a.A) + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
+    AT *dst1 = dst0 + (size_t)NF * a.M;
 
 #pragma unroll 1
     for (int sig = 0; sig < 3; sig++) {
@@ -115,8 +139,8 @@ __global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwd
                     xa = cmul(xa, w);
                     xb = cmul(xb, w);
                 }
-                dst0[sig * plane + (size_t)f1 * a.M] = xa;
-                if (has1) dst1[sig * plane + (size_t)f1 * a.M] = xb;
+                AElem<A16>::store(dst0 + sig * plane + (size_t)f1 * a.M, xa);
+                if (has1) AElem<A16>::store(dst1 + sig * plane + (size_t)f1 * a.M, xb);
             }
         }
     }
@@ -127,9 +151,9 @@ __global__ void __launch_bounds__(256, R <= 16 ? 4 : 1) spectre_rows_fwd(RowsFwd
 // multiples of 64).  Work items are (tile, signal) with tiles of 8 t2 x 64
 // channels; a persistent block computes one item from a shared-memory stage
 // while cp.async copies the next item's 16 x 8 row segments (64 bf16 each)
-// into the other stage.  Rows are padded to 80 values so the warp's 4 t2 x 8
-// channel-pair reads fall on 32 different banks.  Thread mapping, arithmetic
-// and stores are those of spectre_rows_fwd.
+// into the other stage.  Rows are padded to 72 values so the warp's 8 t2 x 4
+// channel-pair reads fall on 32 different banks.  Arithmetic and stores are
+// those of spectre_rows_fwd.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
@@ -141,38 +165,81 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ void cp_async16_rows(void *smem_dst, const void *src) {
+// 16-byte copy of a streamed input row segment, marked first to leave L2 (so
+// the row pass's reads do not push A, which the slice pass reads next, out of
+// L2)
+__device__ __forceinline__ void cp_async16_rows(void *smem_dst, const void *src, uint64_t pol) {
+#if SPECTRE_L2_HINTS
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;"
+                 :
+                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src), "l"(pol)
+                 : "memory");
+#else
+    (void)pol;
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
                  :
                  : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
                  : "memory");
+#endif
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// one bf16 (re, im) pair of A, kept in L2 for the slice pass
+__device__ __forceinline__ void store_a16_keep(__nv_bfloat162 *p, float2 v, uint64_t pol) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+#if SPECTRE_L2_HINTS
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;"
+                 :
+                 : "l"(p), "r"(*reinterpret_cast<const uint32_t *>(&h)), "l"(pol)
+                 : "memory");
+#else
+    (void)pol;
+    *p = h;
+#endif
 }
 
-constexpr int kFwdPipeRow = 80;                          // bf16 per padded row
+constexpr int kFwdPipeRow = 72;                          // bf16 per padded row (36 words)
 constexpr int kFwdPipeStage = 16 * 8 * kFwdPipeRow / 2;  // 4-byte words per stage
 
+template <bool A16>
 __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
     constexpr int R = 16, NF = R / 2 + 1;
+    using AT = typename AElem<A16>::T;
     extern __shared__ float4 smem_f4[];
     uint32_t *stage0 = reinterpret_cast<uint32_t *>(smem_f4);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t2l = (warp & 1) * 4 + (lane & 3);           // 0..7
-    const int cpl = (warp >> 1) * 8 + (lane >> 2);         // 0..31
+    // a warp covers 8 consecutive t2 x 4 channel pairs (lane = t2l + 8 (cpl % 4)),
+    // so each of its stores to A is 8 consecutive t2 of one channel and slice
+    // (a 32-byte sector for bf16 A); with 36-word rows the stage reads hit
+    // bank 4 t2l + cpl mod 32, all different
+    const int t2l = lane & 7;                              // 0..7
+    const int cpl = warp * 4 + (lane >> 3);                // 0..31
     const int ntg = a.M / 8, ncg = a.Cw / 64;
-    const long long nitems = 3LL * ntg * ncg * a.B;
+    const int nitems = 3 * ntg * ncg * a.B;                // < 2^31 (checked by the launcher)
     const size_t rowstep = (size_t)a.M * a.C;
     const size_t plane = (size_t)a.B * a.Cw * NF * a.M;
 
-    // item = ((b * ncg + cg) * ntg + tg) * 3 + sig
-    auto decode = [&](long long item, int &sig, int &tg, int &cg, int &b) {
-        sig = (int)(item % 3);
-        long long r = item / 3;
-        tg = (int)(r % ntg);
-        r /= ntg;
-        cg = (int)(r % ncg);
-        b = (int)(r / ncg);
+    // item = ((b * ncg + cg) * ntg + tg) * 3 + sig, decoded with 32-bit
+    // multiply-high division by the launch's fixed divisors
+    auto decode = [&](int item, int &sig, int &tg, int &cg, int &b) {
+        const uint32_t r1 = fdiv((uint32_t)item, a.fd3);
+        sig = item - 3 * (int)r1;
+        const uint32_t r2 = fdiv(r1, a.fd_ntg);
+        tg = (int)r1 - ntg * (int)r2;
+        const uint32_t r3 = fdiv(r2, a.fd_ncg);
+        cg = (int)r2 - ncg * (int)r3;
+        b = (int)r3;
     };
-    auto prefetch = [&](long long item, int st) {
+    const uint64_t pol_in = l2_evict_first(), pol_a = l2_evict_last();
+    auto prefetch = [&](int item, int st) {
         int sig, tg, cg, b;
         decode(item, sig, tg, cg, b);
         uint32_t *dst = stage0 + st * kFwdPipeStage;
@@ -182,16 +249,16 @@ __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
         for (int i = tid; i < 16 * 8 * 8; i += 256) {       // (t1, t2 row, 16-byte piece)
             const int piece = i & 7, rr = i >> 3, t1 = rr >> 3, tr = rr & 7;
             cp_async16_rows(dst + rr * (kFwdPipeRow / 2) + 4 * piece,
-                            base + (size_t)t1 * rowstep + (size_t)tr * a.C + 8 * piece);
+                            base + (size_t)t1 * rowstep + (size_t)tr * a.C + 8 * piece, pol_in);
         }
     };
 
-    long long it = blockIdx.x;
+    int it = blockIdx.x;
     if (it < nitems) prefetch(it, 0);
     cp_async_commit();
 #pragma unroll 1
     for (int k = 0; it < nitems; k++, it += gridDim.x) {
-        const long long nxt = it + gridDim.x;
+        const int nxt = it + gridDim.x;
         if (nxt < nitems) prefetch(nxt, (k + 1) & 1);
         cp_async_commit();
         cp_async_wait1();
@@ -208,8 +275,8 @@ __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
             z[t1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
         }
         Dft<R>::run(z);
-        float2 *dst0 = a.A + sig * plane + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
-        float2 *dst1 = dst0 + (size_t)NF * a.M;
+        AT *dst0 = static_cast<AT *>(a.A) + sig * plane + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
+        AT *dst1 = dst0 + (size_t)NF * a.M;
 #pragma unroll
         for (int f1 = 0; f1 < NF; f1++) {
             float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
@@ -221,8 +288,13 @@ __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
                 xa = cmul(xa, w);
                 xb = cmul(xb, w);
             }
-            dst0[(size_t)f1 * a.M] = xa;
-            dst1[(size_t)f1 * a.M] = xb;
+            if constexpr (A16) {
+                store_a16_keep(dst0 + (size_t)f1 * a.M, xa, pol_a);
+                store_a16_keep(dst1 + (size_t)f1 * a.M, xb, pol_a);
+            } else {
+                AElem<A16>::store(dst0 + (size_t)f1 * a.M, xa);
+                AElem<A16>::store(dst1 + (size_t)f1 * a.M, xb);
+            }
         }
         // every read of this stage is done before it is refilled
         __syncthreads();
@@ -308,17 +380,19 @@ template <int M> struct SliceCfg {
 // Forward M-point transform of one slice of A.  On return thread j holds
 // X[j + r NT], r < RL, in x[].  buf must not be in use by other threads'
 // loads (callers separate uses with a barrier).
-template <int M>
-__device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bool live, float2 *buf,
-                                              const SliceTables &tb, int j, float2 (&x)[SliceCfg<M>::RL]) {
+template <int M, bool A16>
+__device__ __forceinline__ void slice_forward(const typename AElem<A16>::T *__restrict__ src, bool live,
+                                              float2 *buf, const SliceTables &tb, int j,
+                                              float2 (&x)[SliceCfg<M>::RL]) {
     using Cfg = SliceCfg<M>;
+    using AE = AElem<A16>;
     constexpr int NP = Cfg::NP, NT = Cfg::NT;
     if constexpr (NP == 0) {
-        x[0] = live ? __ldg(src) : make_float2(0.f, 0.f);
+        x[0] = live ? AE::load(src) : make_float2(0.f, 0.f);
     } else if constexpr (NP == 1) {
         constexpr int R = Cfg::RL;
 #pragma unroll
-        for (int r = 0; r < R; r++) x[r] = live ? __ldg(src + j + r * NT) : make_float2(0.f, 0.f);
+        for (int r = 0; r < R; r++) x[r] = live ? AE::load(src + j + r * NT) : make_float2(0.f, 0.f);
         Dft<R>::run(x);
     } else {
         // first pass: global -> registers -> smem (Ns = 1, no twiddle)
@@ -331,7 +405,7 @@ __device__ __forceinline__ void slice_forward(const float2 *__restrict__ src, bo
             if (NBF % NT == 0 || bf < NBF) {
                 float2 v[R];
 #pragma unroll
-                for (int r = 0; r < R; r++) v[r] = live ? __ldg(src + bf + r * NBF) : make_float2(0.f, 0.f);
+                for (int r = 0; r < R; r++) v[r] = live ? AE::load(src + bf + r * NBF) : make_float2(0.f, 0.f);
                 Dft<R>::run(v);
 #pragma unroll
                 for (int r = 0; r < R; r++) buf[spad(bf * R + r)] = v[r];
@@ -456,10 +530,12 @@ __device__ __forceinline__ void slice_inverse_store(float2 (&o)[SliceCfg<M>::RL]
     }
 }
 
-template <int M>
+template <int M, bool A16>
 __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spectre_slices(SliceArgs a) {
     using Cfg = SliceCfg<M>;
+    using AT = typename AElem<A16>::T;
     constexpr int NT = Cfg::NT, RL = Cfg::RL, PROD = Cfg::PROD;
+    static_assert(!(A16 && PROD == kProdGlobal), "the product is parked in fp32 A");
     extern __shared__ float4 smem_f4[];
     const int sl = threadIdx.x / NT;
     const int j = threadIdx.x % NT;
@@ -477,7 +553,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     const int c = a.c_lo + (int)(bcl % a.Cw);
     const int h = c / a.D;
     const size_t sig_stride = (size_t)a.B * a.Cw * NF * M;
-    const float2 *srcA = a.A + (size_t)bcl * NF * M + (size_t)f1 * M;
+    const AT *srcA = static_cast<const AT *>(a.A) + (size_t)bcl * NF * M + (size_t)f1 * M;
     PStore ps;
     if (a.p16) {
         const size_t pslice = p16_pair_slice(b, c, f1, a.C, NF);
@@ -499,7 +575,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     // each thread owns bins f = f1 + R (j + r NT), r < RL, of the product;
     // with kProdGlobal S is parked in this slice's q row of A, which nothing
     // reads once the q transform has passed its first stage
-    float2 *park = const_cast<float2 *>(srcA);
+    float2 *park = A16 ? nullptr : reinterpret_cast<float2 *>(const_cast<AT *>(srcA));
     auto put = [&](int r, float2 v) {
         if constexpr (PROD == kProdSmem) sbuf[j + r * NT] = v;
         else if constexpr (PROD == kProdRegs) s[r] = v;
@@ -512,7 +588,7 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     };
 
     // q: S = Q * G' / L
-    slice_forward<M>(srcA, live, buf, a.tabs, j, x);
+    slice_forward<M, A16>(srcA, live, buf, a.tabs, j, x);
 #pragma unroll
     for (int r = 0; r < RL; r++) {
         int f = f1 + a.R * (j + r * NT);
@@ -529,12 +605,12 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
     }
     if constexpr (Cfg::NP >= 2) __syncthreads();
     // k: S *= conj(K)
-    slice_forward<M>(srcA + sig_stride, live, buf, a.tabs, j, x);
+    slice_forward<M, A16>(srcA + sig_stride, live, buf, a.tabs, j, x);
 #pragma unroll
     for (int r = 0; r < RL; r++) put(r, cmulc(get(r), x[r]));
     if constexpr (Cfg::NP >= 2) __syncthreads();
     // v: O = S * V
-    slice_forward<M>(srcA + 2 * sig_stride, live, buf, a.tabs, j, x);
+    slice_forward<M, A16>(srcA + 2 * sig_stride, live, buf, a.tabs, j, x);
 #pragma unroll
     for (int r = 0; r < RL; r++) x[r] = cmul(get(r), x[r]);
     slice_inverse_store<M>(x, buf, a.tabs, j, ps, a.twL, f1);
@@ -888,15 +964,15 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     const int tl = tid & 1, cp = tid >> 1, c0 = 2 * cp;
     const bool live = cp < CP;
     const int npair_cols = a.M / T2C;
-    const long long ngroups = (long long)a.B * npair_cols;
+    const int ngroups = a.B * npair_cols;   // < 2^31 (checked by the launcher)
     const uint4 *P4 = static_cast<const uint4 *>(a.P);       // one uint4 = 2 columns of a pair
     const float2 *ps2 = reinterpret_cast<const float2 *>(a.pscale);
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
     const int rowstep = a.M * C;
 
-    auto prefetch = [&](long long grp, int st) {
-        const int b = (int)(grp / npair_cols), t2 = (int)(grp % npair_cols) * T2C;
+    auto prefetch = [&](int grp, int st) {
+        const int b = grp / npair_cols, t2 = (grp - b * npair_cols) * T2C;
         uint32_t *pst = stage0 + st * stage_words;
         uint32_t *xst = pst + NF * CP * 4;
         for (int i = tid; i < NF * CP; i += nthr) {            // i = f1 * CP + pair
@@ -917,19 +993,19 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     const float g1 = live ? __ldg(a.gamma + c0 + 1) : 0.f, be1 = live ? __ldg(a.beta + c0 + 1) : 0.f;
     const float invC = 1.0f / (float)C;
     const bool pre = NV && (a.norm & 1), rms = NV && ((a.norm >> 1) & 1);   // residual after the norm; RMSNorm
-    long long grp = blockIdx.x;
+    int grp = blockIdx.x;
     if (grp < ngroups) prefetch(grp, 0);
     cp_async_commit();
 #pragma unroll 1
     for (int k = 0; grp < ngroups; k++, grp += gridDim.x) {
-        const long long nxt = grp + gridDim.x;
+        const int nxt = grp + gridDim.x;
         if (nxt < ngroups) prefetch(nxt, (k + 1) & 1);
         cp_async_commit();
         cp_async_wait1();
         __syncthreads();
         const uint32_t *pst = stage0 + (k & 1) * stage_words;
         const uint32_t *xst = pst + NF * CP * 4;
-        const int b = (int)(grp / npair_cols), t2 = (int)(grp % npair_cols) * T2C + tl;
+        const int b = grp / npair_cols, t2 = (grp - b * npair_cols) * T2C + tl;
         float z0[R], z1[R], s[R];
         {
             float2 Z[R];
@@ -1032,24 +1108,30 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
 // launchers
 // ---------------------------------------------------------------------------
 template <int R>
-static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a, cudaStream_t s) {
-    if (R == 16 && dtype == 1 && a.vec2 && a.C % 8 == 0 && a.c_lo % 64 == 0 && a.Cw % 64 == 0 &&
-        a.M % 8 == 0) {
+static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a0, cudaStream_t s) {
+    const long long pipe_items = 3LL * (a0.M / 8) * (a0.Cw / 64) * a0.B;
+    if (R == 16 && dtype == 1 && a0.vec2 && a0.C % 8 == 0 && a0.c_lo % 64 == 0 && a0.Cw % 64 == 0 &&
+        a0.M % 8 == 0 && pipe_items < (1LL << 31)) {
+        RowsFwdArgs a = a0;
+        a.fd3 = make_fastdiv(3);
+        a.fd_ntg = make_fastdiv((uint32_t)(a.M / 8));
+        a.fd_ncg = make_fastdiv((uint32_t)(a.Cw / 64));
         const size_t smem = (size_t)2 * kFwdPipeStage * 4;
+        auto k = a.a16 ? spectre_rows_fwd_pipe<true> : spectre_rows_fwd_pipe<false>;
         int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spectre_rows_fwd_pipe, 256, smem) !=
-                cudaSuccess || per_sm < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1)
             per_sm = 1;
-        const long long nitems = 3LL * (a.M / 8) * (a.Cw / 64) * a.B;
         const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
-        spectre_rows_fwd_pipe<<<(unsigned)(nitems < cap ? nitems : cap), 256, smem, s>>>(a);
+        k<<<(unsigned)(pipe_items < cap ? pipe_items : cap), 256, smem, s>>>(a);
         return cudaGetLastError();
     }
-    dim3 grid((a.M + 7) / 8, (a.Cw + 63) / 64, a.B);
+    dim3 grid((a0.M + 7) / 8, (a0.Cw + 63) / 64, a0.B);
     if (dtype == 0)
-        spectre_rows_fwd<R, float><<<grid, 256, 0, s>>>(a);
+        a0.a16 ? spectre_rows_fwd<R, float, true><<<grid, 256, 0, s>>>(a0)
+               : spectre_rows_fwd<R, float, false><<<grid, 256, 0, s>>>(a0);
     else
-        spectre_rows_fwd<R, __nv_bfloat16><<<grid, 256, 0, s>>>(a);
+        a0.a16 ? spectre_rows_fwd<R, __nv_bfloat16, true><<<grid, 256, 0, s>>>(a0)
+               : spectre_rows_fwd<R, __nv_bfloat16, false><<<grid, 256, 0, s>>>(a0);
     return cudaGetLastError();
 }
 
@@ -1068,7 +1150,12 @@ static cudaError_t slices_M(const SliceArgs &a, cudaStream_t s) {
     using Cfg = SliceCfg<M>;
     size_t smem = (size_t)Cfg::SMEM;
     long long nblk = (a.nslices + Cfg::SPB - 1) / Cfg::SPB;
-    auto k = spectre_slices<M>;
+    auto k = spectre_slices<M, false>;
+    if constexpr (Cfg::PROD != kProdGlobal) {
+        if (a.a16) k = spectre_slices<M, true>;
+    } else {
+        if (a.a16) return cudaErrorInvalidValue;   // the product is parked in fp32 A
+    }
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<(unsigned)nblk, Cfg::THREADS, smem, s>>>(a);
     return cudaGetLastError();
@@ -1093,6 +1180,17 @@ cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s) {
         SPECTRE_SLICE_LENGTHS(X)
 #undef X
     default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int M> static bool parks_M() { return SliceCfg<M>::PROD == kProdGlobal; }
+
+bool slice_parks_in_A(int M) {
+    switch (M) {
+#define X(m) case m: return parks_M<m>();
+        SPECTRE_SLICE_LENGTHS(X)
+#undef X
+    default: return false;
     }
 }
 
@@ -1129,7 +1227,8 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
 template <int R, typename T, bool NV>
 static cudaError_t rows_inv_RTV(const RowsInvArgs &a, cudaStream_t s) {
     if constexpr (R == 16 && std::is_same<T, __nv_bfloat16>::value) {
-        if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0) {
+        if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0 &&
+            (long long)a.B * (a.M / 2) < (1LL << 31)) {
             const int threads = ((a.C + 31) / 32) * 32;         // 2 columns x C / 2 pairs
             const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32 + 1) * 32 + 64) * 4;
             auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true, NV> : spectre_rows_inv_ln_pipe<false, NV>;

@@ -24,6 +24,25 @@ namespace spectre {
 
 constexpr int kMaxPasses = 6;
 
+// Division by a divisor fixed for a launch, for numerators n < 2^31:
+// q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
+// m = floor(2^32 (2^s - d) / d) + 1 (exact on that range; the sum stays
+// below 2^32).  Work-item decoding uses it instead of 64-bit division.
+struct FastDiv {
+    uint32_t d, m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    f.s = 0;
+    while ((1ull << f.s) < d) f.s++;
+    f.m = (uint32_t)((((1ull << 32) * ((1ull << f.s) - d)) / d) + 1);
+    return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    return (__umulhi(n, f.m) + n) >> f.s;
+}
+
 // Per-pass twiddle tables of the M-point slice transforms.  Pass p of
 // direction d (0 = forward radix order, 1 = reversed) with radix R_p and
 // stride Ns_p (product of the earlier radices) uses
@@ -34,12 +53,15 @@ struct SliceTables {
 
 struct RowsFwdArgs {
     const void *q, *k, *v;
-    float2 *A;            // [3][B][Cw][R/2+1][M]: channels c_lo .. c_lo + Cw - 1
+    void *A;              // [3][B][Cw][R/2+1][M]: channels c_lo .. c_lo + Cw - 1;
+                          // float2, or __nv_bfloat162 (re, im) with a16
+    int a16;
     const float2 *twL;    // exp(-2 pi i e / L), e in [0, L/2]
     int B, L, M, C;
     int c_lo, Cw;         // channel wave (c_lo even)
     int vec2;             // C even: load channel pairs as one vector
     int nsm;              // multiprocessors (grid of the persistent variant)
+    FastDiv fd3, fd_ntg, fd_ncg;   // set by the launcher of the persistent variant
 };
 
 // fp16 P (bf16 I/O) interleaves the two channels c = 2 cp, 2 cp + 1 of a pair:
@@ -51,7 +73,8 @@ __host__ __device__ inline size_t p16_pair_slice(int b, int c, int f1, int C, in
 }
 
 struct SliceArgs {
-    const float2 *A;      // [3][B][Cw][R/2+1][M]: the wave's channels
+    const void *A;        // [3][B][Cw][R/2+1][M]: the chunk's channels, float2 or (a16) bf16 pairs
+    int a16;
     void *P;              // float2 [B][C][NF][M], or __half2 pair-interleaved (p16_pair_slice)
     float *pscale;        // p16: P = stored * pscale, pair-interleaved like P
     const float2 *twL;
@@ -67,6 +90,7 @@ struct SliceArgs {
     const void *w64op;    // DFT-64 / 64 as a 128 x 128 fp16 operand (canonical layout)
     int *err;             // device error word: bit 0 = a tensor-core wait timed out,
                           // bit 1 = a slice exceeded the tensor-memory product budget
+    int test_stall;       // wait-timeout test: block 0 of the tensor-core pass issues no MMA
     long long nslices;    // B * Cw * (R/2+1)
     float invL;
 };
@@ -161,6 +185,9 @@ __host__ __device__ inline int dft64_operand_offset(int n, int k) {
 
 // whether M is a supported slice length (2^k <= 16384 or 3*2^k <= 12288)
 bool slice_length_supported(int M);
+// whether the CUDA-core slice pass for M parks its running product in A (fp32
+// A required)
+bool slice_parks_in_A(int M);
 // threads per slice and slices per block the slice kernel uses for M
 void slice_geometry(int M, int *threads_per_slice, int *slices_per_block, size_t *smem_bytes);
 

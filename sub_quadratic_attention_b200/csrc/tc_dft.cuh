@@ -88,6 +88,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase, uint32_
     return false;
 }
 
+// Arrive on the mbarrier (one of its expected arrivals) and add `bytes` to
+// the transaction count its current phase waits for.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" : : "r"(mbar), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk asynchronous copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory, completing as
+// transaction bytes on the mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :
+        : "r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" : : "r"(base), "r"(ncols)
                  : "memory");

@@ -7,9 +7,13 @@ L x L mixing matrix is circulant; §2.3: truncation keeps bins f < F).
 * out is linear in each of q, k, v (exactly, for a power-of-two scale);
 
 Shifted runs differ from the unshifted one by rounding only.  With bf16 I/O
-the slice-pass output P is stored in fp16 under a per-slice power-of-two
-scale: relative rounding error <= 2^-11 per value, about 4e-4 rms between two
-runs, so the shift checks allow 1e-3 there and 2e-5 for fp32 I/O (fp32 P).
+the row-pass output A is stored as bf16 pairs (relative rounding <= 2^-9 per
+value, about 1.1e-3 rms per transformed signal; three signals enter the
+product, so about 2e-3 rms per run) and the slice-pass output P in fp16 under
+a per-slice power-of-two scale (2^-11).  Two runs round different values, so
+they differ by about sqrt(2) x 2.3e-3 = 3.2e-3 (measured on B200 for both
+bf16 workloads); the shift checks allow 6e-3 there, still below the 1e-2 bar
+each run must meet against the oracle, and 2e-5 for fp32 I/O (fp32 A and P).
 * q = k = v = cos(2 pi a t / L) gives out = (L^2 / 4) G[a] cos(2 pi a t / L)
   when a < F and 0 otherwise.
 """
@@ -46,7 +50,7 @@ def test_shift_and_scale_invariants(name):
     e["q"] = torch.roll(d["q"], s, 1)
     e["k"] = torch.roll(d["k"], s, 1)
     same = _out(w, e)
-    tol = 1e-3 if w.dtype == "bf16" else 2e-5
+    tol = 6e-3 if w.dtype == "bf16" else 2e-5
     assert rel_l2(same.cpu().numpy(), base.double().cpu().numpy()) < tol
     e = dict(d)
     e["v"] = torch.roll(d["v"], s, 1)
