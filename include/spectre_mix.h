@@ -201,7 +201,16 @@ enum spectre_option {
      * flight: the run's y is NaN and spectre_mix_device_status reports
      * SPECTRE_ERR_TIMEOUT.  No effect on plans that take the CUDA-core slice
      * pass. */
-    SPECTRE_OPT_TEST_WAIT_TIMEOUT = 4
+    SPECTRE_OPT_TEST_WAIT_TIMEOUT = 4,
+    /* 0 (default): the row pass (the first stage of the forward transforms)
+     * runs on the CUDA cores.  1: plans with bf16 I/O, R = 16 and a channel
+     * count that is a multiple of 64 run it on the tensor cores: one TMA box
+     * per 16 t2 x 64 channels, the 16-point DFT over t1 as bf16 MMAs with the
+     * DFT matrix split into two bf16 terms (so the transform is accurate to
+     * about 2^-17), fp32 accumulation in tensor memory.  Same results within
+     * rounding; measured slower on B200 for the bf16 long workload (36 us
+     * against 25 us per 128-channel launch), so it is off by default. */
+    SPECTRE_OPT_ROW_TENSOR_CORES = 5
 };
 
 enum spectre_norm {

@@ -33,7 +33,8 @@ struct dct_mix_s {
     float eps;
     int device;
     int nsm;
-    float2 *tables;   // twN[d] = exp(-2 pi i j / d), then tq[d] = exp(-i pi k / (2d))
+    float2 *tables;   // twN[d] = exp(-2 pi i j / d), tq[d] = exp(-i pi k / (2d)), then the
+                      // lane-major tables tl1[E][32], tl2[5][32], tl3[E][32] (E = d / 32)
     void *stage;      // dct_mix_run_host staging
     size_t stage_bytes;
 };
@@ -56,6 +57,10 @@ struct Args {
     float *mix;
     const float2 *twN;
     const float2 *tq;
+    // lane-major copies, so that a warp's table load is one contiguous 256-byte
+    // access: tl1[k][l] = w_N^{l k}; tl2[s][l] = the lane-stage twiddle
+    // w_{2h}^{l mod h} of stage h = 16 >> s; tl3[k][l] = tq[k + E brev5(l)]
+    const float2 *tl1, *tl2, *tl3;
 };
 
 template <typename T> struct Row;
@@ -122,17 +127,17 @@ template <> struct RegDft<32> {
 // Forward N-point FFT of the warp's N values.  On entry lane l, register r
 // holds z[l + 32 r]; on exit it holds Z[r + E * brev5(l)].
 template <int N>
-__device__ __forceinline__ void fft_forward(float2 (&v)[N / 32], int lane, const float2 *twN) {
+__device__ __forceinline__ void fft_forward(float2 (&v)[N / 32], int lane, const Args &a) {
     constexpr int E = N / 32;
-    RegDft<E>::run(v, twN);
+    RegDft<E>::run(v, a.twN);
 #pragma unroll
-    for (int k = 1; k < E; k++) v[k] = cmul(v[k], __ldg(twN + lane * k));
+    for (int k = 1; k < E; k++) v[k] = cmul(v[k], __ldg(a.tl1 + 32 * k + lane));
     // 32-point DFT across lanes, radix-2 decimation in frequency: at stage h
     // the lanes l and l ^ h form a butterfly with twiddle w_{2h}^{l mod h}.
 #pragma unroll
-    for (int h = 16; h >= 1; h >>= 1) {
+    for (int h = 16, st = 0; h >= 1; h >>= 1, st++) {
         const bool up = (lane & h) != 0;
-        const float2 t = __ldg(twN + (lane & (h - 1)) * (16 / h) * E);
+        const float2 t = __ldg(a.tl2 + 32 * st + lane);
 #pragma unroll
         for (int k = 0; k < E; k++) {
             const float2 p = shfl_xor2(v[k], h);
@@ -146,12 +151,12 @@ __device__ __forceinline__ void fft_forward(float2 (&v)[N / 32], int lane, const
 // E-point DFT's adjoint conj(DFT(conj(.))).  Layouts swap: in, register r of
 // lane l holds Y[r + E * brev5(l)]; out, it holds N * y[l + 32 r].
 template <int N>
-__device__ __forceinline__ void fft_adjoint(float2 (&v)[N / 32], int lane, const float2 *twN) {
+__device__ __forceinline__ void fft_adjoint(float2 (&v)[N / 32], int lane, const Args &a) {
     constexpr int E = N / 32;
 #pragma unroll
-    for (int h = 1; h <= 16; h <<= 1) {
+    for (int h = 1, st = 4; h <= 16; h <<= 1, st--) {
         const bool up = (lane & h) != 0;
-        const float2 t = cconj(__ldg(twN + (lane & (h - 1)) * (16 / h) * E));
+        const float2 t = cconj(__ldg(a.tl2 + 32 * st + lane));
 #pragma unroll
         for (int k = 0; k < E; k++) {
             const float2 p = shfl_xor2(v[k], h);
@@ -159,10 +164,10 @@ __device__ __forceinline__ void fft_adjoint(float2 (&v)[N / 32], int lane, const
         }
     }
 #pragma unroll
-    for (int k = 1; k < E; k++) v[k] = cmul(v[k], cconj(__ldg(twN + lane * k)));
+    for (int k = 1; k < E; k++) v[k] = cmul(v[k], cconj(__ldg(a.tl1 + 32 * k + lane)));
 #pragma unroll
     for (int k = 0; k < E; k++) v[k] = cconj(v[k]);
-    RegDft<E>::run(v, twN);
+    RegDft<E>::run(v, a.twN);
 #pragma unroll
     for (int k = 0; k < E; k++) v[k] = cconj(v[k]);
 }
@@ -183,19 +188,24 @@ struct Entropy {
 // Frequency f of the pair (rows a, b) with Zf = Z[f], Zp = Z[N - f] (Z[0]
 // for f = 0): the DCT coefficients c[f] (entropy), then the filtered and
 // re-twiddled spectrum Y[f] = V'_a[f] + i V'_b[f] of the inverse.
+// ws: the filter w in shared memory, entry i at i + i / 32 (one pad word per
+// 32: the bit-reversed frequencies of a warp's lanes fall on distinct banks)
 template <int N>
-__device__ __forceinline__ float2 spectrum(float2 Zf, float2 Zp, int f, const Args &a, Entropy &en) {
+__device__ __forceinline__ float2 spectrum(float2 Zf, float2 Zp, int k, int lane, const Args &a,
+                                           const float *ws, Entropy &en) {
+    constexpr int E = N / 32;
+    const int f = k + E * (int)(__brev((unsigned)lane) >> 27);
     // the two real rows' FFTs: V_a = (Zf + conj Zp) / 2, V_b = (Zf - conj Zp) / 2i
     const float2 Va = make_float2(0.5f * (Zf.x + Zp.x), 0.5f * (Zf.y - Zp.y));
     const float2 Vb = make_float2(0.5f * (Zf.y + Zp.y), 0.5f * (Zp.x - Zf.x));
-    const float2 q = __ldg(a.tq + f);     // (cos, -sin)(pi f / 2N)
+    const float2 q = __ldg(a.tl3 + 32 * k + lane);     // (cos, -sin)(pi f / 2N)
     const float cf = q.x, sf = -q.y;
     // c[f] = Re(e^{-i pi f/2N} V[f]); c[N-f] = Re(e^{-i pi (N-f)/2N} conj V[f])
     const float caf = cf * Va.x + sf * Va.y, cap = sf * Va.x - cf * Va.y;
     const float cbf = cf * Vb.x + sf * Vb.y, cbp = sf * Vb.x - cf * Vb.y;
     en.add(caf, cbf, (f == 0 ? 1.0f : 2.0f) / (float)N);
-    const float wf = __ldg(a.w + f);
-    const float wp = f == 0 ? 0.0f : __ldg(a.w + (N - f));   // c[N] = 0 for f = 0
+    const float wf = ws[f + (f >> 5)];
+    const float wp = f == 0 ? 0.0f : ws[(N - f) + ((N - f) >> 5)];   // c[N] = 0 for f = 0
     const float gaf = caf * wf, gap = cap * wp, gbf = cbf * wf, gbp = cbp * wp;
     // V'[f] = e^{i pi f/2N} (g[f] - i g[N-f])
     const float2 Pa = make_float2(cf * gaf + sf * gap, sf * gaf - cf * gap);
@@ -219,6 +229,9 @@ __global__ void __launch_bounds__(256, dct_blocks_per_sm<N>()) dct_mix_kernel(Ar
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
     const T *X = static_cast<const T *>(a.x);
     T *Y = static_cast<T *>(a.y);
+    __shared__ float ws[N + N / 32];
+    for (int i = threadIdx.x; i < N; i += blockDim.x) ws[i + (i >> 5)] = __ldg(a.w + i);
+    __syncthreads();
 
     for (long long pr = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; pr < npairs;
          pr += nwarps) {
@@ -243,27 +256,27 @@ __global__ void __launch_bounds__(256, dct_blocks_per_sm<N>()) dct_mix_kernel(Ar
 #pragma unroll
         for (int r = H2; r < E; r++) v[r] = shfl_xor2(od[E - 1 - r], 31);
 
-        fft_forward<N>(v, lane, a.twN);
+        fft_forward<N>(v, lane, a);
 
         // register k of lane l holds Z[f], f = k + E * mrev; Z[N - f] sits in
         // register E-k of lane l^31 (k > 0) or register 0 of lane src0 (k = 0)
         Entropy en;
         {
             const float2 zp = shfl2(v[0], src0);
-            v[0] = spectrum<N>(v[0], zp, E * mrev, a, en);
+            v[0] = spectrum<N>(v[0], zp, 0, lane, a, ws, en);
         }
 #pragma unroll
         for (int k = 1; k <= E / 2; k++) {
             if (k < E - k) {
                 const float2 pk = shfl_xor2(v[E - k], 31);
                 const float2 pj = shfl_xor2(v[k], 31);
-                const float2 yk = spectrum<N>(v[k], pk, k + E * mrev, a, en);
-                const float2 yj = spectrum<N>(v[E - k], pj, E - k + E * mrev, a, en);
+                const float2 yk = spectrum<N>(v[k], pk, k, lane, a, ws, en);
+                const float2 yj = spectrum<N>(v[E - k], pj, E - k, lane, a, ws, en);
                 v[k] = yk;
                 v[E - k] = yj;
             } else {   // k = E/2 pairs with itself across lanes
                 const float2 pk = shfl_xor2(v[k], 31);
-                v[k] = spectrum<N>(v[k], pk, k + E * mrev, a, en);
+                v[k] = spectrum<N>(v[k], pk, k, lane, a, ws, en);
             }
         }
 
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(256, dct_blocks_per_sm<N>()) dct_mix_kernel(Ar
             a.route[ta + 1] = Hb <= a.tau ? 1 : 0;
         }
 
-        fft_adjoint<N>(v, lane, a.twN);
+        fft_adjoint<N>(v, lane, a);
 
         // m[2n] = u[n], m[2n+1] = u[N-1-n] with u = adjoint / N; lane l owns
         // n = l + 32 q, and u[N-1-n] is register E-1-q of lane 31-l
@@ -401,6 +414,9 @@ int run(dct_mix_s *h, long long T, const void *x, const float *w, const float *g
     a.mix = mix;
     a.twN = h->tables;
     a.tq = h->tables + h->d;
+    a.tl1 = h->tables + 2 * h->d;
+    a.tl2 = a.tl1 + h->d;          // E x 32 = d entries
+    a.tl3 = a.tl2 + 5 * 32;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = h->dtype == SPECTRE_F32
                               ? launch_T<float>(h->d, a, debug, h->nsm, s)
@@ -428,12 +444,26 @@ int dct_mix_create(dct_mix_t *out, int d, int dtype, float eps) {
         return SPECTRE_ERR_DEVICE;
     }
     if (major != 10) return SPECTRE_ERR_DEVICE;
-    std::vector<float2> tab(2 * (size_t)d);
+    // twN, tq, then the lane-major tl1 [E][32], tl2 [5][32], tl3 [E][32]
+    const int E = d / 32;
+    std::vector<float2> tab(4 * (size_t)d + 5 * 32);
     for (int j = 0; j < d; j++) {
         const double ang = 2.0 * M_PI * (double)j / (double)d;
         tab[j] = make_float2((float)std::cos(ang), (float)-std::sin(ang));
         const double half = M_PI * (double)j / (2.0 * (double)d);
         tab[d + j] = make_float2((float)std::cos(half), (float)-std::sin(half));
+    }
+    float2 *tl1 = tab.data() + 2 * d, *tl2 = tl1 + d, *tl3 = tl2 + 5 * 32;
+    for (int k = 0; k < E; k++)
+        for (int l = 0; l < 32; l++) {
+            tl1[32 * k + l] = tab[(size_t)((l * k) % d)];
+            int rev = 0;
+            for (int bit = 0; bit < 5; bit++) rev |= ((l >> bit) & 1) << (4 - bit);
+            tl3[32 * k + l] = tab[d + k + E * rev];
+        }
+    for (int st = 0; st < 5; st++) {
+        const int hh = 16 >> st;
+        for (int l = 0; l < 32; l++) tl2[32 * st + l] = tab[(size_t)((l & (hh - 1)) * (16 / hh) * E)];
     }
     dct_mix_s *h = new (std::nothrow) dct_mix_s();
     if (!h) return SPECTRE_ERR_NOMEM;

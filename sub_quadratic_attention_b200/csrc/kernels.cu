@@ -19,9 +19,14 @@
 
 #include "fft_regs.cuh"
 #include "kernels.cuh"
+#include "tc_dft.cuh"
 
 #ifndef SPECTRE_L2_HINTS
 #define SPECTRE_L2_HINTS 1
+#endif
+// token columns per group of the prefetching inverse pass (1 or 2)
+#ifndef SPECTRE_INV_COLS
+#define SPECTRE_INV_COLS 2
 #endif
 
 namespace spectre {
@@ -268,6 +273,9 @@ __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
         const uint32_t *stg = stage0 + (k & 1) * kFwdPipeStage;
         const int t2 = tg * 8 + t2l;
         const int cl = 64 * cg + 2 * cpl;                  // channel within the chunk
+        // w_L^{t2}, loaded before the transform; w_L^{f1 t2} follow as its powers
+        // (seven products in fp32 add far less than bf16's rounding)
+        const float2 wt = __ldg(a.twL + t2);
         float2 z[R];
 #pragma unroll
         for (int t1 = 0; t1 < R; t1++) {
@@ -277,17 +285,16 @@ __global__ void __launch_bounds__(256, 4) spectre_rows_fwd_pipe(RowsFwdArgs a) {
         Dft<R>::run(z);
         AT *dst0 = static_cast<AT *>(a.A) + sig * plane + ((size_t)b * a.Cw + cl) * NF * a.M + t2;
         AT *dst1 = dst0 + (size_t)NF * a.M;
+        // wh = w_L^{f1 t2} / 2 and wb = -i wh: channel a = (Z_f + conj Z_{R-f}) wh,
+        // channel b = (Z_f - conj Z_{R-f}) wb
+        float2 wh = make_float2(0.5f, 0.f);
 #pragma unroll
         for (int f1 = 0; f1 < NF; f1++) {
-            float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
-            float2 xa = cscale(cadd(zf, zc), 0.5f);
-            float2 d = csub(zf, zc);
-            float2 xb = make_float2(0.5f * d.y, -0.5f * d.x);
-            if (f1 > 0) {
-                float2 w = __ldg(a.twL + f1 * t2);
-                xa = cmul(xa, w);
-                xb = cmul(xb, w);
-            }
+            if (f1 > 0) wh = cmul(wh, wt);
+            const float2 wb = make_float2(wh.y, -wh.x);
+            const float2 zf = z[f1], zc = cconj(z[(R - f1) % R]);
+            const float2 xa = cmul(cadd(zf, zc), wh);
+            const float2 xb = cmul(csub(zf, zc), wb);
             if constexpr (A16) {
                 store_a16_keep(dst0 + (size_t)f1 * a.M, xa, pol_a);
                 store_a16_keep(dst1 + (size_t)f1 * a.M, xb, pol_a);
@@ -940,20 +947,33 @@ __global__ void __launch_bounds__(1024) spectre_rows_inv_ln_reg(RowsInvArgs a) {
 // spectre_rows_inv_ln_reg with T2C = 2.
 // ---------------------------------------------------------------------------
 constexpr int kInvPipeMaxC = 512;
+constexpr uint32_t kInvWaitLimit = 1u << 12;   // polls of up to 1 ms each
 
-// shared-memory words of one stage: P [NF][CP][2 columns] as uint2 (the pair's
-// two half2), then x [16 rows][2 columns][C + 32] bf16
-__host__ __device__ inline int inv_pipe_stage_words(int C) {
-    return 9 * (C / 2) * 2 * 2 + 16 * 2 * (C + 32) / 2;
+// shared-memory words of one stage: P [NF][CP][T2C columns] as uint2 (the
+// pair's two half2), then x [16 rows][T2C columns][C + 32] bf16
+__host__ __device__ inline int inv_pipe_stage_words(int C, int T2C) {
+    return 9 * (C / 2) * T2C * 2 + 16 * T2C * (C + 32) / 2;
 }
 
-template <bool DEBUG_OUT, bool NV>
-__global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(RowsInvArgs a) {
-    constexpr int R = 16, NF = R / 2 + 1, T2C = 2;
+// Before a 16-byte or 8-byte cp.async of P: T2C = 2 takes both columns of a
+// pair slice in one 16-byte piece, T2C = 1 its one column's 8 bytes.
+__device__ __forceinline__ void cp_async8(void *smem_dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;"
+                 :
+                 : "r"((uint32_t)__cvta_generic_to_shared(smem_dst)), "l"(src)
+                 : "memory");
+}
+
+// T2C token columns per group: 2 (blocks of C threads, one per SM) or 1
+// (blocks of C / 2 threads, two per SM, so one block's LayerNorm barriers
+// overlap the other block's work)
+template <bool DEBUG_OUT, bool NV, int T2C>
+__global__ void __launch_bounds__(kInvPipeMaxC * T2C / 2, 2 / T2C) spectre_rows_inv_ln_pipe(RowsInvArgs a) {
+    constexpr int R = 16, NF = R / 2 + 1;
     extern __shared__ float4 smem_f4[];
     const int C = a.C, CP = C / 2, XS = C + 32;
     const int nthr = blockDim.x, nwarps = nthr >> 5;
-    const int stage_words = inv_pipe_stage_words(C);
+    const int stage_words = inv_pipe_stage_words(C, T2C);
     uint32_t *stage0 = reinterpret_cast<uint32_t *>(smem_f4);
     // per-warp partial sums as [T2C * R rows][nwarps + 1] (padded: distinct
     // banks for the writes and the per-row reads), then stat[2][T2C][R]
@@ -961,7 +981,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     float *part = reinterpret_cast<float *>(stage0 + 2 * stage_words);
     float *stat = part + T2C * R * PS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tl = tid & 1, cp = tid >> 1, c0 = 2 * cp;
+    const int tl = tid & (T2C - 1), cp = tid / T2C, c0 = 2 * cp;
     const bool live = cp < CP;
     const int npair_cols = a.M / T2C;
     const int ngroups = a.B * npair_cols;   // < 2^31 (checked by the launcher)
@@ -970,22 +990,39 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(a.y);
     const int rowstep = a.M * C;
+    // one mbarrier per stage for its x rows (bulk copies)
+    uint64_t *xbar = reinterpret_cast<uint64_t *>(stat + 2 * T2C * R);
+    if (tid == 0) {
+        tc::mbar_init(tc::smem_u32(xbar), 1);
+        tc::mbar_init(tc::smem_u32(xbar + 1), 1);
+    }
+    __syncthreads();
+    const uint32_t xrow_bytes = (uint32_t)C * 2;
 
+    // P: 16-byte cp.async pieces (per channel pair and f1: both columns' two
+    // fp16 complex values); x: the stage's 2 x 16 token rows, one bulk copy
+    // of C bf16 per row, issued by the lanes of warp 0
     auto prefetch = [&](int grp, int st) {
         const int b = grp / npair_cols, t2 = (grp - b * npair_cols) * T2C;
         uint32_t *pst = stage0 + st * stage_words;
-        uint32_t *xst = pst + NF * CP * 4;
+        uint32_t *xst = pst + NF * CP * 2 * T2C;
         for (int i = tid; i < NF * CP; i += nthr) {            // i = f1 * CP + pair
-            const int f1 = i / CP, pr = i - f1 * CP;
+            const int f1 = (int)fdiv((uint32_t)i, a.fd_cp), pr = i - f1 * CP;
             const size_t slice = ((size_t)b * CP + pr) * NF + f1;
-            cp_async16(pst + 4 * i, P4 + (slice * a.M + t2) / 2);
+            if constexpr (T2C == 2)
+                cp_async16(pst + 4 * i, P4 + (slice * a.M + t2) / 2);
+            else
+                cp_async8(pst + 2 * i, static_cast<const uint2 *>(a.P) + slice * a.M + t2);
         }
-        const __nv_bfloat16 *xb = x + ((size_t)b * a.L + t2) * C;
-        const int chunks = C / 8;                              // 16-byte pieces per row
-        for (int i = tid; i < R * T2C * chunks; i += nthr) {   // i = (t1 * 2 + col) * chunks + k
-            const int rowi = i / chunks, k = i - rowi * chunks;
-            const int t1 = rowi >> 1, col = rowi & 1;
-            cp_async16(xst + rowi * (XS / 2) + 4 * k, xb + (size_t)t1 * rowstep + (size_t)col * C + 8 * k);
+        if (warp == 0) {
+            const uint32_t mb = tc::smem_u32(xbar + st);
+            if (lane == 0) tc::mbar_arrive_expect_tx(mb, R * T2C * xrow_bytes);
+            __syncwarp();
+            if (lane < R * T2C) {
+                const int t1 = lane / T2C, col = lane & (T2C - 1);   // lane = row t1 T2C + col
+                const __nv_bfloat16 *src = x + ((size_t)b * a.L + t2 + col + (size_t)t1 * a.M) * C;
+                tc::bulk_copy_g2s(tc::smem_u32(xst + lane * (XS / 2)), src, xrow_bytes, mb);
+            }
         }
     };
 
@@ -996,15 +1033,24 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
     int grp = blockIdx.x;
     if (grp < ngroups) prefetch(grp, 0);
     cp_async_commit();
+    bool late = false;      // a bounded wait for x rows gave up
+    int done = grp;         // first group not finished
+    int nissued = grp < ngroups ? 1 : 0;   // x fills issued / waited for (fill n: stage n & 1, phase (n >> 1) & 1)
+    int nwaited = 0;
 #pragma unroll 1
     for (int k = 0; grp < ngroups; k++, grp += gridDim.x) {
         const int nxt = grp + gridDim.x;
-        if (nxt < ngroups) prefetch(nxt, (k + 1) & 1);
+        if (nxt < ngroups) {
+            prefetch(nxt, (k + 1) & 1);
+            nissued++;
+        }
         cp_async_commit();
         cp_async_wait1();
-        __syncthreads();
+        if (tc::mbar_wait(tc::smem_u32(xbar + (k & 1)), (k >> 1) & 1, kInvWaitLimit)) nwaited++;
+        else late = true;
+        if (__syncthreads_or(late)) break;
         const uint32_t *pst = stage0 + (k & 1) * stage_words;
-        const uint32_t *xst = pst + NF * CP * 4;
+        const uint32_t *xst = pst + NF * CP * 2 * T2C;
         const int b = grp / npair_cols, t2 = (grp - b * npair_cols) * T2C + tl;
         float z0[R], z1[R], s[R];
         {
@@ -1013,7 +1059,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
             auto ld2 = [&](int f1, float2 &pa, float2 &pb) {
                 pa = pb = make_float2(0.f, 0.f);
                 if (!live) return;
-                const uint2 u = reinterpret_cast<const uint2 *>(pst)[(f1 * CP + cp) * 2 + tl];
+                const uint2 u = reinterpret_cast<const uint2 *>(pst)[(f1 * CP + cp) * T2C + tl];
                 const float2 sc = __ldg(ps2 + sa + f1);
                 pa = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.x)), sc.x);
                 pb = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.y)), sc.y);
@@ -1039,7 +1085,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
                 if (DEBUG_OUT && live)
                     *reinterpret_cast<float2 *>(a.out_f32 + (tok0 + (size_t)t1 * a.M) * C + c0) =
                         make_float2(z0[t1], z1[t1]);
-                const uint32_t xw = (live && !pre) ? xst[(t1 * 2 + tl) * (XS / 2) + cp] : 0u;
+                const uint32_t xw = (live && !pre) ? xst[(t1 * T2C + tl) * (XS / 2) + cp] : 0u;
                 const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw));
                 z0[t1] = live ? z0[t1] + xv.x : 0.f;
                 z1[t1] = live ? z1[t1] + xv.y : 0.f;
@@ -1059,12 +1105,12 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
                 }
             }
             {
-                // channel pairs of one column differ in lane bits [1, 5)
+                // channel pairs of one column differ in lane bits [log2 T2C, 5)
                 float v[R];
 #pragma unroll
                 for (int t1 = 0; t1 < R; t1++) v[t1] = s[t1];
                 int row0 = 0;
-                HalvingReduce<R, 1, 5>::run(v, lane, row0);
+                HalvingReduce<R, (T2C == 2 ? 1 : 0), 5>::run(v, lane, row0);
                 part[(tl * R + row0) * PS + warp] = v[0];
             }
             __syncthreads();
@@ -1090,7 +1136,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
                 float y0 = fmaf((z0[t1] - mu) * rstd, g0, be0);
                 float y1 = fmaf((z1[t1] - mu) * rstd, g1, be1);
                 if (pre) {   // the residual, still in this stage
-                    const uint32_t xw = xst[(t1 * 2 + tl) * (XS / 2) + cp];
+                    const uint32_t xw = xst[(t1 * T2C + tl) * (XS / 2) + cp];
                     const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw));
                     y0 += xv.x;
                     y1 += xv.y;
@@ -1100,8 +1146,24 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
         }
         // every read of this stage and of stat is done before the stage is refilled
         __syncthreads();
+        done = grp + gridDim.x;
     }
     cp_async_wait_all();
+    if (__syncthreads_or(late)) {
+        // a copy that never arrived: report it, let this block's own copies
+        // land (bounded), and make y of the groups it did not finish NaN
+        if (tid == 0) {
+            if (a.err) atomicOr(a.err, 1);
+            for (int n = nwaited; n < nissued; n++)
+                tc::mbar_wait(tc::smem_u32(xbar + (n & 1)), (n >> 1) & 1, kInvWaitLimit);
+        }
+        for (int g = done; g < ngroups; g += gridDim.x) {
+            const int b = g / npair_cols, t2 = (g - b * npair_cols) * T2C + tl;
+            if (!live) continue;
+            for (int t1 = 0; t1 < R; t1++)
+                *reinterpret_cast<uint32_t *>(y + ((size_t)b * a.L + t2 + (size_t)t1 * a.M) * C + c0) = 0x7fc07fc0u;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1109,6 +1171,7 @@ __global__ void __launch_bounds__(kInvPipeMaxC, 1) spectre_rows_inv_ln_pipe(Rows
 // ---------------------------------------------------------------------------
 template <int R>
 static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a0, cudaStream_t s) {
+    if (R == 16 && dtype == 1 && a0.row_tc && rows_tc_applies(a0)) return launch_rows_fwd_tc(a0, s);
     const long long pipe_items = 3LL * (a0.M / 8) * (a0.Cw / 64) * a0.B;
     if (R == 16 && dtype == 1 && a0.vec2 && a0.C % 8 == 0 && a0.c_lo % 64 == 0 && a0.Cw % 64 == 0 &&
         a0.M % 8 == 0 && pipe_items < (1LL << 31)) {
@@ -1227,19 +1290,23 @@ static cudaError_t rows_inv_RT(const RowsInvArgs &a, cudaStream_t s) {
 template <int R, typename T, bool NV>
 static cudaError_t rows_inv_RTV(const RowsInvArgs &a, cudaStream_t s) {
     if constexpr (R == 16 && std::is_same<T, __nv_bfloat16>::value) {
-        if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % 2 == 0 &&
-            (long long)a.B * (a.M / 2) < (1LL << 31)) {
-            const int threads = ((a.C + 31) / 32) * 32;         // 2 columns x C / 2 pairs
-            const size_t smem = ((size_t)2 * inv_pipe_stage_words(a.C) + (threads / 32 + 1) * 32 + 64) * 4;
-            auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true, NV> : spectre_rows_inv_ln_pipe<false, NV>;
+        constexpr int T2C = SPECTRE_INV_COLS;
+        if (a.reg_variant && a.C % 8 == 0 && a.C <= kInvPipeMaxC && a.M % T2C == 0 &&
+            (long long)a.B * (a.M / T2C) < (1LL << 31)) {
+            const int threads = ((T2C * (a.C / 2) + 31) / 32) * 32;   // T2C columns x C / 2 pairs
+            const size_t smem =
+                ((size_t)2 * inv_pipe_stage_words(a.C, T2C) + (threads / 32 + 1) * 16 * T2C + 32 * T2C + 4) * 4;
+            auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true, NV, T2C> : spectre_rows_inv_ln_pipe<false, NV, T2C>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             int per_sm = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess ||
                 per_sm < 1)
                 per_sm = 1;
-            const long long ngroups = (long long)a.B * (a.M / 2);
+            const long long ngroups = (long long)a.B * (a.M / T2C);
             const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
-            k<<<(unsigned)(ngroups < cap ? ngroups : cap), threads, smem, s>>>(a);
+            RowsInvArgs ap = a;
+            ap.fd_cp = make_fastdiv((uint32_t)(a.C / 2));
+            k<<<(unsigned)(ngroups < cap ? ngroups : cap), threads, smem, s>>>(ap);
             return cudaGetLastError();
         }
     }

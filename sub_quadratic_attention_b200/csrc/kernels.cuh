@@ -62,6 +62,8 @@ struct RowsFwdArgs {
     int vec2;             // C even: load channel pairs as one vector
     int nsm;              // multiprocessors (grid of the persistent variant)
     FastDiv fd3, fd_ntg, fd_ncg;   // set by the launcher of the persistent variant
+    int *err;             // device error word (tensor-core variant: bit 0 = a bounded wait gave up)
+    int row_tc;           // take the tensor-core variant where it applies
 };
 
 // fp16 P (bf16 I/O) interleaves the two channels c = 2 cp, 2 cp + 1 of a pair:
@@ -109,10 +111,16 @@ struct RowsInvArgs {
     int nsm;              // multiprocessors (grid of the persistent variant)
     int norm;             // bit 0: residual after the norm; bit 1: RMSNorm (no mean)
     float eps;
+    FastDiv fd_cp;        // set by the launcher of the prefetching variant: C / 2
+    int *err;             // device error word (prefetching variant: bit 0 = a bounded wait gave up)
 };
 
 // Returns cudaSuccess or the launch error.  dtype: 0 fp32, 1 bf16.
 cudaError_t launch_rows_fwd(int R, int dtype, const RowsFwdArgs &a, cudaStream_t s);
+// the tensor-core row pass (bf16 in, bf16 A, R = 16; rows_tc.cu) and whether
+// it covers a launch
+bool rows_tc_applies(const RowsFwdArgs &a);
+cudaError_t launch_rows_fwd_tc(const RowsFwdArgs &a, cudaStream_t s);
 cudaError_t launch_slices(const SliceArgs &a, cudaStream_t s);
 cudaError_t launch_slices_mma4096(const SliceArgs &a, cudaStream_t s);
 cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStream_t s);

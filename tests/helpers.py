@@ -19,7 +19,7 @@ def to_device(inputs):
 
 
 def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None, norm=None,
-                complex_gate=False):
+                complex_gate=False, row_tensor_cores=False):
     """Run the CUDA path through the C ABI.  Returns (out_f32 or None, y) on CPU.
     tensor_cores: None keeps the plan's default slice pass, True/False sets it."""
     from sub_quadratic_attention_b200 import binding
@@ -27,7 +27,8 @@ def run_library(w, inputs_cpu, debug=True, stream=None, tensor_cores=None, norm=
 
     d = to_device(inputs_cpu)
     with SpectreMix(w.B, w.L, w.H, w.D, w.F, w.dtype, w.eps, tensor_cores=tensor_cores,
-                    norm=norm, complex_gate=complex_gate) as mix:
+                    norm=norm, complex_gate=complex_gate,
+                    row_tensor_cores=row_tensor_cores) as mix:
         y = torch.empty_like(d["x"])
         out = torch.empty((w.B, w.L, w.C), dtype=torch.float32, device="cuda") if debug else None
         mix(d["q"], d["k"], d["v"], d["x"], d["G"], d["gamma"], d["beta"], y=y, out=out,

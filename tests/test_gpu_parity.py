@@ -239,3 +239,18 @@ def test_blockwise_mode(B, L, H, D, n, F, dtype):
     e_out, e_y = check_parity(wb, out.cpu().view(wb.B, n, C), y.cpu().view(wb.B, n, C),
                               out_ref, y_ref)
     print(f"block mode {B}x{L} n={n}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+@pytest.mark.parametrize("case", ["bf16_long", "mixed_radix_c128", "batch3_c192"])
+def test_row_pass_on_tensor_cores(case):
+    """SPECTRE_OPT_ROW_TENSOR_CORES: the row pass as TMA-fed bf16 MMAs (DFT-16
+    matrix split into two bf16 terms) gives the oracle's result within the bf16
+    bar, at full size and on a mixed-radix plan with B > 1."""
+    w = {"bf16_long": WORKLOADS["bf16_long"],
+         "mixed_radix_c128": custom(2, 12288, 2, 64, 6145, dtype="bf16"),
+         "batch3_c192": custom(3, 4096, 3, 64, 1000, dtype="bf16")}[case]
+    inp = make_inputs(w)
+    out, y = run_library(w, inp, row_tensor_cores=True)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"{case}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
