@@ -24,6 +24,10 @@
 #ifndef SPECTRE_L2_HINTS
 #define SPECTRE_L2_HINTS 1
 #endif
+// cap on the persistent row pass's blocks per multiprocessor
+#ifndef SPECTRE_ROW_CTAS_PER_SM
+#define SPECTRE_ROW_CTAS_PER_SM 4
+#endif
 // token columns per group of the prefetching inverse pass (1 or 2)
 #ifndef SPECTRE_INV_COLS
 #define SPECTRE_INV_COLS 2
@@ -1184,6 +1188,7 @@ static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a0, cudaStream_t s) 
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem) != cudaSuccess || per_sm < 1)
             per_sm = 1;
+        if (per_sm > SPECTRE_ROW_CTAS_PER_SM) per_sm = SPECTRE_ROW_CTAS_PER_SM;
         const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
         k<<<(unsigned)(pipe_items < cap ? pipe_items : cap), 256, smem, s>>>(a);
         return cudaGetLastError();

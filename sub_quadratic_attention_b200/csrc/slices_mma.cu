@@ -62,6 +62,11 @@
 #ifndef SPECTRE_SLICE_PARTS
 #define SPECTRE_SLICE_PARTS 2
 #endif
+// persistent blocks per multiprocessor of the tensor-core slice pass (at most
+// 2: shared memory and tensor memory fit two)
+#ifndef SPECTRE_SLICE_CTAS_PER_SM
+#define SPECTRE_SLICE_CTAS_PER_SM 2
+#endif
 
 namespace spectre {
 namespace {
@@ -604,7 +609,7 @@ cudaError_t launch_slices_mma4096(const SliceArgs &a, cudaStream_t s) {
     const long long nitems = (long long)a.B * ((a.Cw + 1) / 2) * NF;
     if (nitems <= 0) return cudaSuccess;
     if (nitems >= (1LL << 31)) return cudaErrorInvalidValue;
-    const long long cap = (long long)kBlocksPerSM * (a.nsm > 0 ? a.nsm : 148);
+    const long long cap = (long long)SPECTRE_SLICE_CTAS_PER_SM * (a.nsm > 0 ? a.nsm : 148);
     const unsigned grid = (unsigned)(nitems < cap ? nitems : cap);
     if (!a.a16) return cudaErrorInvalidValue;   // the pass reads bf16 A
     constexpr int NP = SPECTRE_SLICE_PARTS;
