@@ -370,13 +370,23 @@ template <int M, int NT, int D, int P, int PEND> struct MidPasses {
 // forward transforms of a slice.
 enum SliceProduct { kProdSmem = 0, kProdRegs = 1, kProdGlobal = 2 };
 
+constexpr int spb_warp_aligned(int nt) {
+    int s = 256 / nt;
+    while (s > 1 && (s * nt) % 32 != 0) s--;
+    return s;
+}
+
 template <int M> struct SliceCfg {
     static constexpr RadList S = make_schedule(M);
     static constexpr int NP = S.n;
     static constexpr int RL = NP > 0 ? S.r[NP - 1] : 1;   // largest radix, last
     static constexpr int R0 = NP > 0 ? S.r[0] : 1;
     static constexpr int NT = M / RL;                      // threads per slice
-    static constexpr int SPB = NT >= 256 ? 1 : 256 / NT;   // slices per block
+    // slices per block: as many as fill 256 threads with a whole number of
+    // warps (M = 768: 4 slices of 48 threads, not 5, whose 240 threads end in
+    // half a warp; measured on B200 for the mixed-radix workload, the slice
+    // pass went from 1.37 to 1.03 ms per step)
+    static constexpr int SPB = NT >= 256 ? 1 : spb_warp_aligned(NT);
     static constexpr int THREADS = NT * SPB;
     static constexpr int BUF = NP >= 2 ? (M + M / 16) : 0; // float2 per slice (padded)
     static constexpr int PROD = (BUF + M) * SPB * 8 <= 72 * 1024 ? kProdSmem
