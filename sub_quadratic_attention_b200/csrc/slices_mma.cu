@@ -24,8 +24,9 @@
 //
 // Truncation prunes the tensor work: the gate is zero outside min(f, L-f) < F,
 // so pass 2 of the forward transforms computes only the k2 groups (8 k2
-// values = one 16-column MMA) that hold a live bin, and pass 1 of the inverse
-// runs only the K steps of those groups.  The product S lives in tensor
+// values = 16 result columns) that hold a live bin, as one chain of 8 MMAs
+// over those groups' DFT-operand rows gathered side by side, and pass 1 of
+// the inverse runs only the K steps of those groups.  The product S lives in tensor
 // memory between the transforms.
 //
 // Scaling: every pass-1 input is scaled by a power of two s with
@@ -77,13 +78,17 @@ constexpr uint32_t kTileLBO = 144;              // K-adjacent core matrices (pad
 constexpr uint32_t kTileSBO = 16 * kTileLBO;    // 8-row groups
 constexpr uint32_t kTileBytes = 16 * kTileSBO;  // 128 rows
 constexpr uint32_t kOpBytes = 128 * 128 * 2;    // DFT-64 operand, LBO 128, SBO 2048
+constexpr uint32_t kGroupOpBytes = 2 * 2048;     // one k2 group's 16 operand rows (two 8-row groups)
+// the operand rows of the item's live k2 groups, side by side, so that pass 2
+// of a forward transform is one 8-MMA chain of N = 16 x (live groups)
+constexpr uint32_t kOp2Bytes = kMmaMaxGroups * kGroupOpBytes;
 constexpr uint32_t kDCols = 128;                // pass results
 constexpr uint32_t kSCols = 16 * kMmaMaxGroups; // the running product S
 constexpr uint32_t kWaitLimit = 1u << 12;       // polls of up to 1 ms each
 constexpr uint32_t kTestWaitLimit = 4;          // the wait-timeout test's block
 constexpr uint32_t kRowBytes = kM * 4;           // one bf16 slice row of A
 constexpr uint32_t kStageBytes = 2 * kRowBytes;  // the two slices of an item
-constexpr size_t kSmemBytes = kTileBytes + kOpBytes + kStageBytes + 64;
+constexpr size_t kSmemBytes = kTileBytes + kOpBytes + kOp2Bytes + kStageBytes + 64;
 
 __device__ __forceinline__ uint32_t tile_off(uint32_t row, uint32_t k) {
     return (row >> 3) * kTileSBO + (k >> 3) * kTileLBO + (row & 7) * 16 + (k & 7) * 2;
@@ -109,7 +114,7 @@ __device__ __forceinline__ int scale_shift(float m) {
 }
 
 struct Mma {
-    uint32_t tile, op, mbar, dcol, phase;
+    uint32_t tile, op, op2, mbar, dcol, phase;
     uint32_t limit;   // polls per wait
     bool late;        // this thread's last wait gave up
     bool no_issue;    // the wait-timeout test: wait without issuing any MMA
@@ -122,7 +127,8 @@ struct Mma {
     // columns, over the K steps (16 reals each) whose bit is set in ksteps.
     // Otherwise all 8 K steps, and for each group g in gmask the 16 result
     // columns of DFT-matrix rows 16 g .. 16 g + 15 (outputs 8 g .. 8 g + 7),
-    // packed side by side from column 0.
+    // packed side by side from column 0: one MMA per K step over the gathered
+    // rows in op2, which hold gmask's groups in ascending order.
     __device__ __forceinline__ bool run(uint32_t ksteps, uint32_t gmask, bool full_n) {
         return run(ksteps, gmask, full_n, [] {});
     }
@@ -137,24 +143,29 @@ struct Mma {
         if (threadIdx.x == 0 && !no_issue) {
             tc::fence_after();
             if (full_n) {
-                uint32_t acc = 0;
-                for (uint32_t km = ksteps; km; km &= km - 1) {
-                    const int ks = __ffs(km) - 1;
-                    tc::mma_f16(dcol, tc::make_desc(tile + ks * 2 * kTileLBO, kTileLBO, kTileSBO),
-                                tc::make_desc(op + ks * 2 * 128, 128, 2048), tc::idesc_f16(128), acc);
-                    acc = 1;
+                const uint64_t da = tc::make_desc(tile, kTileLBO, kTileSBO);
+                const uint64_t db = tc::make_desc(op, 128, 2048);
+                if (ksteps == 0xFFu) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ks++)
+                        tc::mma_f16(dcol, da + ks * (2 * kTileLBO / 16), db + ks * (2 * 128 / 16),
+                                    tc::idesc_f16(128), ks > 0);
+                } else {
+                    uint32_t acc = 0;
+                    for (uint32_t km = ksteps; km; km &= km - 1) {
+                        const int ks = __ffs(km) - 1;
+                        tc::mma_f16(dcol, da + ks * (2 * kTileLBO / 16), db + ks * (2 * 128 / 16),
+                                    tc::idesc_f16(128), acc);
+                        acc = 1;
+                    }
                 }
             } else {
-                uint32_t gi = 0;
-                for (uint32_t gm = gmask; gm; gm &= gm - 1) {
-                    const int g = __ffs(gm) - 1;
-                    for (int ks = 0; ks < 8; ks++)
-                        tc::mma_f16(dcol + 16 * gi,
-                                    tc::make_desc(tile + ks * 2 * kTileLBO, kTileLBO, kTileSBO),
-                                    tc::make_desc(op + 2 * g * 2048 + ks * 2 * 128, 128, 2048),
-                                    tc::idesc_f16(16), ks > 0);
-                    gi++;
-                }
+                const uint32_t idesc = tc::idesc_f16(16 * __popc(gmask));
+                const uint64_t da = tc::make_desc(tile, kTileLBO, kTileSBO);
+                const uint64_t db = tc::make_desc(op2, 128, 2048);
+#pragma unroll
+                for (int ks = 0; ks < 8; ks++)   // the start address sits in the low bits (16-byte units)
+                    tc::mma_f16(dcol, da + ks * (2 * kTileLBO / 16), db + ks * (2 * 128 / 16), idesc, ks > 0);
             }
             tc::commit(mbar);
         }
@@ -259,8 +270,9 @@ __global__ void __launch_bounds__(128 * NP, kBlocksPerSM) spectre_slices_mma4096
     extern __shared__ __align__(1024) unsigned char smem[];
     unsigned char *tile = smem;
     unsigned char *op = smem + kTileBytes;
-    const uint32_t *stage = reinterpret_cast<const uint32_t *>(op + kOpBytes);   // [2][4096] bf16 pairs
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(op + kOpBytes + kStageBytes);  // [0] MMA, [1] stage
+    unsigned char *op2 = op + kOpBytes;
+    const uint32_t *stage = reinterpret_cast<const uint32_t *>(op2 + kOp2Bytes);   // [2][4096] bf16 pairs
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(op2 + kOp2Bytes + kStageBytes);  // [0] MMA, [1] stage
     uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 2);    // [0] D, [1] S
     float *red = reinterpret_cast<float *>(tslot + 2);           // per-warp maxima
 
@@ -296,6 +308,8 @@ __global__ void __launch_bounds__(128 * NP, kBlocksPerSM) spectre_slices_mma4096
     Mma mma;
     mma.tile = tc::smem_u32(tile);
     mma.op = tc::smem_u32(op);
+    mma.op2 = tc::smem_u32(op2);
+    uint32_t op2_mask = 0;   // the groups whose operand rows op2 holds
     mma.mbar = tc::smem_u32(mbar);
     mma.dcol = tslot[0];
     mma.phase = 0;
@@ -384,10 +398,34 @@ __global__ void __launch_bounds__(128 * NP, kBlocksPerSM) spectre_slices_mma4096
             for (int i = 0; i < gi && gm; i++) gm &= gm - 1;
             if (gm) gmine = __ffs(gm) - 1;
         }
+        // gather the live groups' operand rows for pass 2 (the previous
+        // item's MMAs, the last readers, have completed; the first MMA
+        // chain's proxy fence and barrier publish the copy)
+        if (gmask != op2_mask) {
+            for (int i = tid; i < __popc(gmask) * (int)(kGroupOpBytes / 16); i += NT) {
+                const int gk = i / (int)(kGroupOpBytes / 16);
+                uint32_t gm = gmask;
+                for (int j = 0; j < gk; j++) gm &= gm - 1;
+                const int g = __ffs(gm) - 1;
+                reinterpret_cast<uint4 *>(op2)[i] = reinterpret_cast<const uint4 *>(
+                    op + g * kGroupOpBytes)[i - gk * (int)(kGroupOpBytes / 16)];
+            }
+            op2_mask = gmask;
+        }
+        // this thread's gates, issued now and first used in the first pass-2
+        // epilogue, so the loads are in flight through the q transform
+        GateT graw[GJ];
+#pragma unroll
+        for (int j = 0; j < GJ; j++) {
+            const int f = f1 + a.R * (row + 64 * (8 * (gmine < 0 ? 0 : gmine) + jsub + j));
+            const int ff = min(f, a.L - f);
+            const bool on = live && gmine >= 0 && ff < a.F;
+            if constexpr (CG) graw[j] = on ? __ldg(reinterpret_cast<const float2 *>(Gh) + ff) : make_float2(0.f, 0.f);
+            else graw[j] = on ? __ldg(Gh + ff) : 0.f;
+        }
 
         int shift_sum = 0;   // sum of the applied input shifts of the four transforms
         float omax = 0.f;
-        GateT gate[GJ];      // the gates of this thread's pass-2 bins / L (loaded early)
 #pragma unroll 1
         for (int sig = 0; sig < 3 && !abort; sig++) {
             // pass-1 input: row n2 = row holds a[64 n1 + row]; this thread
@@ -437,22 +475,6 @@ __global__ void __launch_bounds__(128 * NP, kBlocksPerSM) spectre_slices_mma4096
                     *reinterpret_cast<uint4 *>(tile + tile_off(trow, 2 * NV * part + 8 * j)) = u;
                 }
             }
-            if (sig == 0) {   // this thread's gates, loaded while the MMAs run
-#pragma unroll
-                for (int j = 0; j < GJ; j++) {
-                    const int f = f1 + a.R * (row + 64 * (8 * (gmine < 0 ? 0 : gmine) + jsub + j));
-                    const int ff = min(f, a.L - f);
-                    const bool on = live && gmine >= 0 && ff < a.F;
-                    if constexpr (CG) {   // conj(G[L - f]) above L/2
-                        float2 gc = on ? __ldg(reinterpret_cast<const float2 *>(Gh) + ff)
-                                       : make_float2(0.f, 0.f);
-                        if (f > a.L - f) gc.y = -gc.y;
-                        gate[j] = cscale(gc, a.invL);
-                    } else {
-                        gate[j] = on ? __ldg(Gh + ff) * a.invL : 0.f;
-                    }
-                }
-            }
             // after the chain's barrier every thread is done with the staged
             // rows: thread 0 stages the next signal, or the next item's q rows
             if (!mma.run(0xFFu, 0, true, [&] {
@@ -478,8 +500,14 @@ __global__ void __launch_bounds__(128 * NP, kBlocksPerSM) spectre_slices_mma4096
                     const float2 X = make_float2(d[2 * j], d[2 * j + 1]);
                     float2 S;
                     if (sig == 0) {
-                        if constexpr (CG) S = cmul(X, gate[j]);
-                        else S = cscale(X, gate[j]);
+                        if constexpr (CG) {   // conj(G[L - f]) above L/2
+                            const int f = f1 + a.R * (row + 64 * (8 * gmine + jsub + j));
+                            float2 gc = graw[j];
+                            if (f > a.L - f) gc.y = -gc.y;
+                            S = cmul(X, cscale(gc, a.invL));
+                        } else {
+                            S = cscale(X, graw[j] * a.invL);
+                        }
                     } else if (sig == 1) {
                         S = cmulc(make_float2(sv[2 * j], sv[2 * j + 1]), X);
                     } else {
