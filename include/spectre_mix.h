@@ -90,7 +90,9 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F,
  *   gamma, beta: device, fp32 [C].
  *   y          : device, [B, L, C] in the plan's dtype; may not alias inputs.
  * Every pointer must be non-null and 16-byte aligned.  One handle must not run
- * on two streams at once: its workspace is shared by all its runs.
+ * on two streams at once: its workspace is shared by all its runs.  Calls on
+ * one handle come from one host thread at a time (the handle keeps the
+ * captured graph of its last pointer set, SPECTRE_OPT_GRAPH).
  */
 int spectre_mix_run(spectre_mix_t h, const void *q, const void *k, const void *v,
                     const void *x, const float *G, const float *gamma,
@@ -210,7 +212,18 @@ enum spectre_option {
      * about 2^-17), fp32 accumulation in tensor memory.  Same results within
      * rounding; measured slower on B200 for the bf16 long workload (36 us
      * against 25 us per 128-channel launch), so it is off by default. */
-    SPECTRE_OPT_ROW_TENSOR_CORES = 5
+    SPECTRE_OPT_ROW_TENSOR_CORES = 5,
+    /* 1 (default): spectre_mix_run (and spectre_mix_run_host) replays the
+     * step's launches as one CUDA graph,
+     * captured at the first run with a given set of tensor pointers (and
+     * again after a pointer or an option changes) on a stream the handle
+     * owns, and launched on the caller's stream.  A capture costs about as
+     * much as instantiating the graph; replays skip the per-launch host work.
+     * A caller's stream that is itself being captured gets the plain
+     * launches.  0: every run enqueues the launches directly.  Runs with
+     * events (spectre_mix_run_profiled) or a debug output never use the
+     * graph. */
+    SPECTRE_OPT_GRAPH = 6
 };
 
 enum spectre_norm {

@@ -32,6 +32,7 @@ SPECTRE_OPT_NORM = 2
 SPECTRE_OPT_COMPLEX_GATE = 3
 SPECTRE_OPT_TEST_WAIT_TIMEOUT = 4
 SPECTRE_OPT_ROW_TENSOR_CORES = 5
+SPECTRE_OPT_GRAPH = 6
 
 # enum spectre_norm, keyed as in the oracle
 SPECTRE_NORM = {"post_ln": 0, "pre_ln": 1, "post_rms": 2, "pre_rms": 3}
@@ -251,7 +252,8 @@ class SpectreMix:
     def __init__(self, B: int, L: int, H: int, D: int, F: Optional[int] = None,
                  dtype: str = "bf16", eps: float = 1e-5, tensor_cores: Optional[bool] = None,
                  norm: Optional[str] = None, complex_gate: bool = False,
-                 block_len: Optional[int] = None, row_tensor_cores: bool = False):
+                 block_len: Optional[int] = None, row_tensor_cores: bool = False,
+                 graph: Optional[bool] = None):
         self.B, self.L, self.H, self.D = B, L, H, D
         self.C = H * D
         if block_len is not None and (block_len < 1 or L % block_len):
@@ -271,6 +273,8 @@ class SpectreMix:
             spectre_mix_set_option(self.handle, SPECTRE_OPT_COMPLEX_GATE, 1)
         if row_tensor_cores:           # the row pass on the tensor cores (where it applies)
             spectre_mix_set_option(self.handle, SPECTRE_OPT_ROW_TENSOR_CORES, 1)
+        if graph is not None:          # None keeps the library's default
+            spectre_mix_set_option(self.handle, SPECTRE_OPT_GRAPH, 1 if graph else 0)
         self._gate_ref = None
 
     def _check_shapes(self, q, k, v, x, G, gamma, beta, y, out):

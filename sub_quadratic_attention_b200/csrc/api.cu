@@ -64,6 +64,13 @@ struct spectre_mix_s {
     // staging for spectre_mix_run_host, allocated on first use
     void *stage;
     size_t stage_bytes;
+    // the step as a CUDA graph (SPECTRE_OPT_GRAPH): captured on `cap` for the
+    // pointer set gkey, replayed on the caller's stream
+    int use_graph;
+    cudaStream_t cap;
+    cudaGraphExec_t gexec;
+    const void *gkey[8];
+    int gvalid;
 };
 
 namespace {
@@ -94,6 +101,12 @@ bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
 // two regions of 64 channels against 0.366 ms with one of 128).
 #ifndef SPECTRE_A_REGIONS
 #define SPECTRE_A_REGIONS 2
+#endif
+// whether a handle replays its launches as a CUDA graph by default
+// (SPECTRE_OPT_GRAPH; measured on B200: the same time for the bf16 long
+// workload, 2-3 % less for the 65-launch mixed-radix step and fp32 mid)
+#ifndef SPECTRE_GRAPH_DEFAULT
+#define SPECTRE_GRAPH_DEFAULT 1
 #endif
 constexpr double kL2Fraction = SPECTRE_L2_FRACTION;
 constexpr int kARegions = SPECTRE_A_REGIONS;
@@ -143,6 +156,8 @@ int check_device(int *dev_out) {
 
 void free_handle(spectre_mix_s *h) {
     if (!h) return;
+    if (h->gexec) cudaGraphExecDestroy(h->gexec);
+    if (h->cap) cudaStreamDestroy(h->cap);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->aux) cudaStreamDestroy(h->aux);
@@ -439,6 +454,7 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
 
     spectre_mix_s *h = new (std::nothrow) spectre_mix_s();
     if (!h) return SPECTRE_ERR_NOMEM;
+    h->use_graph = SPECTRE_GRAPH_DEFAULT;
     h->device = dev;
     h->g = g;
 
@@ -493,6 +509,63 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     return SPECTRE_OK;
 }
 
+// One run as the handle's CUDA graph: captured (on the handle's own stream,
+// so that the caller's stream may be the legacy default stream) when the
+// pointer set or the plan changed since the last capture, then launched on
+// the caller's stream.  A re-capture updates the executable graph in place
+// where the topology allows, else re-instantiates it.
+static int run_graph(spectre_mix_t h, const void *q, const void *k, const void *v, const void *x,
+                     const float *G, const float *gamma, const float *beta, void *y, cudaStream_t s) {
+    const void *key[8] = {q, k, v, x, G, gamma, beta, y};
+    bool same = h->gvalid != 0;
+    for (int i = 0; i < 8 && same; i++) same = key[i] == h->gkey[i];
+    cudaError_t e = cudaSuccess;
+    if (!same) {
+        h->gvalid = 0;
+        if (!h->cap) {
+            e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                h->cap = nullptr;
+                return cuda_status(e);
+            }
+        }
+        e = cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_status(e);
+        }
+        const int rc = launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, h->cap,
+                                   h->aux, h->ev_fork, h->ev_join);
+        cudaGraph_t graph = nullptr;
+        e = cudaStreamEndCapture(h->cap, &graph);
+        if (rc != SPECTRE_OK || e != cudaSuccess) {
+            if (graph) cudaGraphDestroy(graph);
+            cudaGetLastError();
+            return rc != SPECTRE_OK ? rc : cuda_status(e);
+        }
+        if (h->gexec) {
+            cudaGraphExecUpdateResultInfo info;
+            if (cudaGraphExecUpdate(h->gexec, graph, &info) != cudaSuccess) {
+                cudaGetLastError();
+                cudaGraphExecDestroy(h->gexec);
+                h->gexec = nullptr;
+            }
+        }
+        if (!h->gexec) e = cudaGraphInstantiate(&h->gexec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            h->gexec = nullptr;
+            return cuda_status(e);
+        }
+        for (int i = 0; i < 8; i++) h->gkey[i] = key[i];
+        h->gvalid = 1;
+    }
+    e = cudaGraphLaunch(h->gexec, s);
+    return cuda_status(e);
+}
+
 static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v, const void *x,
                     const float *G, const float *gamma, const float *beta, void *y, float *out_f32,
                     void *const *events, void *stream) {
@@ -507,6 +580,16 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
         return SPECTRE_ERR_DEVICE;
     }
     if (fault_requested("launch")) return SPECTRE_ERR_CUDA;
+    if (h->use_graph && !events && !out_f32) {
+        // a caller that is capturing its own graph gets the launches themselves
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess) {
+            cudaGetLastError();
+            cs = cudaStreamCaptureStatusActive;
+        }
+        if (cs == cudaStreamCaptureStatusNone)
+            return run_graph(h, q, k, v, x, G, gamma, beta, y, static_cast<cudaStream_t>(stream));
+    }
     return launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, out_f32, events,
                        static_cast<cudaStream_t>(stream), h->aux, h->ev_fork, h->ev_join);
 }
@@ -642,6 +725,7 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
 
 int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     if (!h) return SPECTRE_ERR_ARG;
+    h->gvalid = 0;   // the plan may change: the next run captures again
     switch (option) {
     case SPECTRE_OPT_TENSOR_CORES:
         if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
@@ -662,6 +746,10 @@ int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
     case SPECTRE_OPT_ROW_TENSOR_CORES:
         if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
         h->g.row_tc = value;
+        return SPECTRE_OK;
+    case SPECTRE_OPT_GRAPH:
+        if (value != 0 && value != 1) return SPECTRE_ERR_ARG;
+        h->use_graph = value;
         return SPECTRE_OK;
     default: return SPECTRE_ERR_ARG;
     }

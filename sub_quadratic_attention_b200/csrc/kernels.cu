@@ -1200,6 +1200,7 @@ static cudaError_t rows_fwd_R(int dtype, const RowsFwdArgs &a0, cudaStream_t s) 
             per_sm = 1;
         if (per_sm > SPECTRE_ROW_CTAS_PER_SM) per_sm = SPECTRE_ROW_CTAS_PER_SM;
         const long long cap = (long long)per_sm * (a.nsm > 0 ? a.nsm : 148);
+        prefer_max_smem(k);
         k<<<(unsigned)(pipe_items < cap ? pipe_items : cap), 256, smem, s>>>(a);
         return cudaGetLastError();
     }
@@ -1313,6 +1314,7 @@ static cudaError_t rows_inv_RTV(const RowsInvArgs &a, cudaStream_t s) {
                 ((size_t)2 * inv_pipe_stage_words(a.C, T2C) + (threads / 32 + 1) * 16 * T2C + 32 * T2C + 4) * 4;
             auto k = a.out_f32 ? spectre_rows_inv_ln_pipe<true, NV, T2C> : spectre_rows_inv_ln_pipe<false, NV, T2C>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            prefer_max_smem(k);
             int per_sm = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess ||
                 per_sm < 1)

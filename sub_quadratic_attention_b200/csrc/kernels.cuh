@@ -126,6 +126,21 @@ cudaError_t launch_slices_mma4096(const SliceArgs &a, cudaStream_t s);
 cudaError_t launch_rows_inv_ln(int R, int dtype, const RowsInvArgs &a, cudaStream_t s);
 
 // Slice-transform schedule for length M (radices ascending, largest last).
+// Shared-memory carveout of the row, slice and inverse kernels.  With
+// SPECTRE_CARVEOUT_MAX every one of them asks for the largest shared-memory
+// share of the L1/shared array, so consecutive kernels of a step need no
+// reconfiguration of it between them.
+#ifndef SPECTRE_CARVEOUT_MAX
+#define SPECTRE_CARVEOUT_MAX 0
+#endif
+template <class K> inline void prefer_max_smem(K k) {
+#if SPECTRE_CARVEOUT_MAX
+    cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+#else
+    (void)k;
+#endif
+}
+
 struct RadList {
     int n;
     int r[kMaxPasses];

@@ -643,6 +643,7 @@ cudaError_t launch_slices_mma4096(const SliceArgs &a, cudaStream_t s) {
     constexpr int NP = SPECTRE_SLICE_PARTS;
     auto k = a.cgate ? spectre_slices_mma4096<true, NP> : spectre_slices_mma4096<false, NP>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    prefer_max_smem(k);
     k<<<grid, 128 * NP, kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
