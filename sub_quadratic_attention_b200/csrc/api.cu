@@ -49,13 +49,24 @@ struct PathBuffers {
     int *err;            // device error word (bit 0: a tensor-core wait timed out)
 };
 
+// Streams of the chunk pipeline: chunk i runs on stream i % n (0: the
+// caller's stream, k > 0: aux[k - 1]), so a region's next chunk follows its
+// previous one in stream order.  ev_fork orders the aux streams after the
+// caller's earlier work; ev_join[k] orders the caller's stream after aux[k].
+constexpr int kMaxRegions = 4;
+struct ChunkStreams {
+    int n = 1;
+    cudaStream_t aux[kMaxRegions - 1] = {};
+    cudaEvent_t ev_fork = nullptr;
+    cudaEvent_t ev_join[kMaxRegions - 1] = {};
+};
+
 struct spectre_mix_s {
     int device;
     PathGeom g;
-    // second stream and fork/join events: the row pass of one channel chunk
-    // overlaps the slice pass of the previous chunk
-    cudaStream_t aux;
-    cudaEvent_t ev_fork, ev_join;
+    // one stream per A region beyond the first, with fork/join events: the
+    // chunks of different regions overlap
+    ChunkStreams cs;
     // device memory owned by the handle
     void *tables;       // twL followed by the slice tables
     void *ws;           // A, P, pscale
@@ -110,6 +121,7 @@ bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
 #endif
 constexpr double kL2Fraction = SPECTRE_L2_FRACTION;
 constexpr int kARegions = SPECTRE_A_REGIONS;
+static_assert(kARegions >= 1 && kARegions <= 4, "one to four A regions");
 
 // L = R * M: R-point row transforms, M-point slice transforms.
 bool choose_split(int L, int *R, int *M) {
@@ -158,9 +170,11 @@ void free_handle(spectre_mix_s *h) {
     if (!h) return;
     if (h->gexec) cudaGraphExecDestroy(h->gexec);
     if (h->cap) cudaStreamDestroy(h->cap);
-    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-    if (h->ev_join) cudaEventDestroy(h->ev_join);
-    if (h->aux) cudaStreamDestroy(h->aux);
+    if (h->cs.ev_fork) cudaEventDestroy(h->cs.ev_fork);
+    for (int i = 0; i < kMaxRegions - 1; i++) {
+        if (h->cs.ev_join[i]) cudaEventDestroy(h->cs.ev_join[i]);
+        if (h->cs.aux[i]) cudaStreamDestroy(h->cs.aux[i]);
+    }
     if (h->tables) cudaFree(h->tables);
     if (h->ws) cudaFree(h->ws);
     if (h->stage) cudaFree(h->stage);
@@ -321,34 +335,35 @@ bool uses_mma(const PathGeom &g) { return g.tc_mode == 1 && g.mma_ok; }
 // The launch sequence of one mix: per channel chunk the row pass then the
 // slice pass, then the inverse row pass with residual + LayerNorm.  With one
 // A region the chunks run one after another on `s` and each overwrites the
-// previous chunk's A (still in L2).  With two regions the chunks alternate
-// between `s` and `aux` (and between the regions), so the row pass of chunk
-// k + 1 can run while the slice pass of chunk k does; `aux` forks from and
-// joins back into `s`.  events (nullable, one per launch + 1) are recorded
-// before every launch and after the last; with events the schedule is
-// single-stream.
+// previous chunk's A (still in L2).  With n regions (and cs with n streams)
+// chunk i uses region i % n on stream i % n, so the row passes of up to n - 1
+// later chunks can run while a chunk's slice pass does, and a region is
+// rewritten only after its previous chunk's slice pass (stream order).  The
+// aux streams fork from and join back into `s`.  events (nullable, one per
+// launch + 1) are recorded before every launch and after the last; with
+// events the schedule is single-stream.
 int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const void *k, const void *v,
                 const void *x, const float *G, const float *gamma, const float *beta, void *y,
-                float *out_f32, void *const *events, cudaStream_t s, cudaStream_t aux,
-                cudaEvent_t ev_fork, cudaEvent_t ev_join) {
+                float *out_f32, void *const *events, cudaStream_t s, const ChunkStreams *cs) {
     int ev = 0;
     auto mark = [&](cudaStream_t st) -> cudaError_t {
         return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), st) : cudaSuccess;
     };
     const int chunk = g.chunk;
-    const bool two = aux && !events && g.regions == 2;
+    const int nst = (cs && !events && cs->n == g.regions) ? g.regions : 1;
     const size_t region_elems = (size_t)3 * g.B * chunk * g.NF * g.M;
     const size_t elem = g.a16 ? 4 : 8;
     cudaError_t e = cudaSuccess;
-    if (two) {
-        e = cudaEventRecord(ev_fork, s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(aux, ev_fork, 0);
+    if (nst > 1) {
+        e = cudaEventRecord(cs->ev_fork, s);
+        for (int i = 0; i < nst - 1 && e == cudaSuccess; i++) e = cudaStreamWaitEvent(cs->aux[i], cs->ev_fork, 0);
         if (e != cudaSuccess) return cuda_status(e);
     }
     int idx = 0;
     for (int c_lo = 0; c_lo < g.C; c_lo += chunk, idx++) {
         const int Cw = g.C - c_lo < chunk ? g.C - c_lo : chunk;
-        cudaStream_t st = (two && (idx & 1)) ? aux : s;
+        const int si = nst > 1 ? idx % nst : 0;
+        cudaStream_t st = si == 0 ? s : cs->aux[si - 1];
         // this chunk's region of A: [3][B][Cw][NF][M]
         void *A = static_cast<char *>(bf.A) + (size_t)(idx % g.regions) * region_elems * elem;
         RowsFwdArgs fa;
@@ -386,9 +401,9 @@ int launch_path(const PathGeom &g, const PathBuffers &bf, const void *q, const v
         if (e == cudaSuccess) e = launch_slices(sa, st);
         if (e != cudaSuccess) return cuda_status(e);
     }
-    if (two) {
-        e = cudaEventRecord(ev_join, aux);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_join, 0);
+    for (int i = 0; i < nst - 1; i++) {
+        e = cudaEventRecord(cs->ev_join[i], cs->aux[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, cs->ev_join[i], 0);
         if (e != cudaSuccess) return cuda_status(e);
     }
     RowsInvArgs ia;
@@ -495,10 +510,13 @@ int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F, in
     h->bufs.pscale = reinterpret_cast<float *>(base + g.a_bytes + g.p_bytes);
     h->bufs.err = reinterpret_cast<int *>(base + g.a_bytes + g.p_bytes + g.s_bytes - 256);
     e = cudaMemset(h->bufs.err, 0, sizeof(int));
-    if (e == cudaSuccess && g.regions == 2) {
-        e = cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    if (e == cudaSuccess && g.regions > 1) {
+        e = cudaEventCreateWithFlags(&h->cs.ev_fork, cudaEventDisableTiming);
+        for (int i = 0; i < g.regions - 1 && e == cudaSuccess; i++) {
+            e = cudaStreamCreateWithFlags(&h->cs.aux[i], cudaStreamNonBlocking);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->cs.ev_join[i], cudaEventDisableTiming);
+        }
+        if (e == cudaSuccess) h->cs.n = g.regions;
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -536,7 +554,7 @@ static int run_graph(spectre_mix_t h, const void *q, const void *k, const void *
             return cuda_status(e);
         }
         const int rc = launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, h->cap,
-                                   h->aux, h->ev_fork, h->ev_join);
+                                   &h->cs);
         cudaGraph_t graph = nullptr;
         e = cudaStreamEndCapture(h->cap, &graph);
         if (rc != SPECTRE_OK || e != cudaSuccess) {
@@ -591,7 +609,7 @@ static int run_impl(spectre_mix_t h, const void *q, const void *k, const void *v
             return run_graph(h, q, k, v, x, G, gamma, beta, y, static_cast<cudaStream_t>(stream));
     }
     return launch_path(h->g, h->bufs, q, k, v, x, G, gamma, beta, y, out_f32, events,
-                       static_cast<cudaStream_t>(stream), h->aux, h->ev_fork, h->ev_join);
+                       static_cast<cudaStream_t>(stream), &h->cs);
 }
 
 int spectre_mix_run(spectre_mix_t h, const void *q, const void *k, const void *v, const void *x,
@@ -719,8 +737,7 @@ int spectre_mix_run_noalloc(int B, int L, int H, int D, int F, int dtype, float 
     e = launch_make_tables(tw, tl.segs, s);
     if (e != cudaSuccess) return cuda_status(e);
     // single stream: this path creates no streams or events
-    return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s, nullptr, nullptr,
-                       nullptr);
+    return launch_path(g, bf, q, k, v, x, G, gamma, beta, y, nullptr, nullptr, s, nullptr);
 }
 
 int spectre_mix_set_option(spectre_mix_t h, int option, int value) {
