@@ -642,6 +642,86 @@ __global__ void __launch_bounds__(SliceCfg<M>::THREADS, SliceCfg<M>::MINB_C) spe
 // ---------------------------------------------------------------------------
 // NV: the plan uses a norm variant (residual after the norm, or RMSNorm);
 // without it the default LayerNorm(out + x) code is compiled alone.
+// The R = 64 inverse row transform of spectre_rows_inv_ln over two lanes per
+// (column, channel pair).  Every lane of the block runs the same number of
+// iterations (padded with idle items), so the exchange is a full-warp shuffle.
+template <typename T, bool P16>
+__device__ __forceinline__ void inv64_pairs(const RowsInvArgs &a, float *zbuf, int T2C, int ZS, int b, int t2base,
+                                            int CP) {
+    constexpr int R = 64, NF = R / 2 + 1;
+    const int items = 2 * T2C * CP;
+    const int h = threadIdx.x & 1;
+    const int rounds = (items + blockDim.x - 1) / blockDim.x;
+    for (int k = 0; k < rounds; k++) {
+        const int it = threadIdx.x + k * blockDim.x;
+        const int rest = it >> 1;
+        const int tl = rest % T2C, cp = rest / T2C;
+        const int t2 = t2base + tl;
+        const bool ok = it < items && t2 < a.M;
+        const int c0 = 2 * cp;
+        const bool has1 = ok && c0 + 1 < a.C;
+        const size_t sa = ok ? (P16 ? p16_pair_slice(b, c0, 0, a.C, NF) : ((size_t)b * a.C + c0) * NF) : 0;
+        const size_t sb = sa + NF;
+        auto ld2 = [&](int f1, float2 &pa, float2 &pb) {
+            pa = pb = make_float2(0.f, 0.f);
+            if (!ok) return;
+            if constexpr (P16) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(a.P) + (sa + f1) * a.M + t2);
+                const float2 sc = __ldg(reinterpret_cast<const float2 *>(a.pscale) + sa + f1);
+                pa = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.x)), sc.x);
+                if (has1) pb = cscale(__half22float2(*reinterpret_cast<const __half2 *>(&u.y)), sc.y);
+            } else {
+                pa = __ldg(static_cast<const float2 *>(a.P) + (sa + f1) * a.M + t2);
+                if (has1) pb = __ldg(static_cast<const float2 *>(a.P) + (sb + f1) * a.M + t2);
+            }
+        };
+        // v[m] = Z[2 m + h], where Z[f1] = P_a + i P_b and Z[64 - f1] =
+        // conj(P_a) + i conj(P_b) for 0 < f1 < 32, both stored conjugated, and
+        // Z[0], Z[32] keep the real parts only.  Lane h reads P[f1] for f1 = 2 q
+        // + h: Z[f1] is v[q], Z[64 - f1] is v[32 - q - h] (both of parity h).
+        float2 v[32];
+#pragma unroll
+        for (int q = 0; q <= 16; q++) {
+            if (q == 16 && h == 1) break;   // f1 = 33: none
+            const int f1 = 2 * q + h;
+            float2 pv, qv;
+            ld2(f1, pv, qv);
+            if (h == 0 && (q == 0 || q == 16)) {
+                v[q] = make_float2(pv.x, -qv.x);
+            } else {
+                v[q] = make_float2(pv.x - qv.y, -(pv.y + qv.x));
+                const float2 sec = make_float2(pv.x + qv.y, pv.y - qv.x);
+                if (h == 0) {
+                    if (q >= 1 && q <= 15) v[32 - q] = sec;
+                } else {
+                    v[31 - q] = sec;
+                }
+            }
+        }
+        Dft<32>::run(v);
+        // odd lane: W[t] = w64^t O[t]; then lane 0 forms E + W (t < 32),
+        // lane 1 E - W (t + 32)
+#pragma unroll
+        for (int t = 1; t < 32; t++)
+            if (h == 1) v[t] = cmul(v[t], c_w64[t]);
+        float *zr = zbuf + (size_t)tl * ZS + c0;
+#pragma unroll
+        for (int t = 0; t < 32; t++) {
+            const float rx = __shfl_xor_sync(0xffffffffu, v[t].x, 1);
+            const float ry = __shfl_xor_sync(0xffffffffu, v[t].y, 1);
+            const float2 o = h == 0 ? make_float2(v[t].x + rx, v[t].y + ry) : make_float2(rx - v[t].x, ry - v[t].y);
+            if (ok) {
+                // inverse result = conj: real part -> channel c0, imaginary -> c0 + 1
+                float *p = zr + (size_t)(t + 32 * h) * T2C * ZS;
+                if (has1)
+                    *reinterpret_cast<float2 *>(p) = make_float2(o.x, -o.y);
+                else
+                    p[0] = o.x;
+            }
+        }
+    }
+}
+
 template <int R, typename T, bool DEBUG_OUT, bool NV>
 __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
     constexpr int NF = R / 2 + 1;
@@ -652,6 +732,13 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
     const int b = blockIdx.y;
     const int t2base = blockIdx.x * T2C;
     const int CP = (a.C + 1) / 2;
+    if constexpr (R == 64) {
+        // two lanes per (column, channel pair): lane h of an even/odd pair takes
+        // the even (h = 0) or odd (h = 1) inputs Z[2m + h], a 32-point DFT each;
+        // then DFT64[t] = E[t] + w64^t O[t] and DFT64[t + 32] = E[t] - w64^t O[t],
+        // lane 0 forming t < 32 and lane 1 t >= 32 after one exchange
+        inv64_pairs<T, P16>(a, zbuf, T2C, ZS, b, t2base, CP);
+    } else {
     const int items = T2C * CP;
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
         const int tl = it % T2C, cp = it / T2C;
@@ -704,6 +791,7 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
                 p[0] = Z[t1].x;
         }
     }
+    }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nw = blockDim.x >> 5;
@@ -719,6 +807,50 @@ __global__ void __launch_bounds__(512) spectre_rows_inv_ln(RowsInvArgs a) {
         const T *xr = x + tok * a.C;
         T *yr = y + tok * a.C;
         float *zr = zbuf + (size_t)row * ZS;
+        if (a.vec2) {   // channel pairs: 2-wide loads and stores (ZS is even, C even)
+            float2 *zr2 = reinterpret_cast<float2 *>(zr);
+            const int C2 = a.C / 2;
+            float s = 0.f;
+            for (int c = lane; c < C2; c += 32) {
+                const float2 o = zr2[c];
+                if (DEBUG_OUT) *reinterpret_cast<float2 *>(a.out_f32 + tok * a.C + 2 * c) = o;
+                float2 z = o;
+                if (!pre) {
+                    const float2 xv = Elem<T>::load2(xr + 2 * c);
+                    z.x += xv.x;
+                    z.y += xv.y;
+                }
+                zr2[c] = z;
+                s = rms ? fmaf(z.x, z.x, fmaf(z.y, z.y, s)) : s + (z.x + z.y);
+            }
+            float mean = 0.f, rstd;
+            if (rms) {
+                rstd = rsqrtf(warp_sum(s) * invC + a.eps);
+            } else {
+                mean = warp_sum(s) * invC;
+                float ss = 0.f;
+                for (int c = lane; c < C2; c += 32) {
+                    const float2 z = zr2[c];
+                    const float d0 = z.x - mean, d1 = z.y - mean;
+                    ss = fmaf(d0, d0, fmaf(d1, d1, ss));
+                }
+                rstd = rsqrtf(warp_sum(ss) * invC + a.eps);
+            }
+            for (int c = lane; c < C2; c += 32) {
+                const float2 z = zr2[c];
+                const float2 g = __ldg(reinterpret_cast<const float2 *>(a.gamma) + c);
+                const float2 bb = __ldg(reinterpret_cast<const float2 *>(a.beta) + c);
+                float y0 = fmaf((z.x - mean) * rstd, g.x, bb.x);
+                float y1 = fmaf((z.y - mean) * rstd, g.y, bb.y);
+                if (pre) {
+                    const float2 xv = Elem<T>::load2(xr + 2 * c);
+                    y0 += xv.x;
+                    y1 += xv.y;
+                }
+                Elem<T>::store2(yr + 2 * c, y0, y1);
+            }
+            continue;
+        }
         float s = 0.f;
         for (int c = lane; c < a.C; c += 32) {
             float o = zr[c];

@@ -254,3 +254,18 @@ def test_row_pass_on_tensor_cores(case):
     out_ref, y_ref = oracle_full(w, inp)
     e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
     print(f"{case}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+@pytest.mark.parametrize("case,dtype", [((1, 2 ** 20, 1, 8, 65536), "bf16"), ((1, 2 ** 20, 1, 4, 100000), "f32"),
+                                        ((1, 786432, 1, 4, 50000), "bf16"), ((1, 2 ** 20, 1, 2, 2 ** 19 + 1), "f32")])
+def test_longest_slices_parked_product(case, dtype):
+    """Slices of 16384 and 12288 points (R = 64), whose running product is
+    parked in the q row of fp32 A: truncations whose edge falls on a row of
+    bins (F = 65536) or inside one (F = 100000), a 12288-point slice, and
+    every bin kept (F = L/2 + 1)."""
+    w = custom(*case, dtype=dtype)
+    inp = make_inputs(w)
+    out, y = run_library(w, inp)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"longest slices {w.name} {dtype}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
