@@ -101,11 +101,17 @@ bool fault_requested(const char *what) {
 
 bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
 
-// Fraction of L2 that one chunk's A (or both regions' A) may fill.  Measured
-// on B200: data written by one kernel is read back by the next entirely from
-// L2 up to about 64 MB (of 126 MB); at 96 MB about 40 MB comes from DRAM.
+// Fraction of L2 that all regions' A together may fill.  Measured on B200:
+// data written by one kernel and read back by the next comes entirely from
+// L2 up to about 64 MB (of 126 MB) when nothing else streams through; in the
+// mix the region being read is the one written one chunk earlier, and with
+// 0.9 (two regions of 128 channels, 113 MB, for the bf16 long workload) the
+// slice passes still read only 5 MB of DRAM per step.  0.9 against 0.45 (two
+// regions of 64 channels): 0.3256 against 0.3297 ms per mix for the bf16 long
+// workload, 1.420 against 1.435 ms for the mixed-radix one, the same time for
+// the others.
 #ifndef SPECTRE_L2_FRACTION
-#define SPECTRE_L2_FRACTION 0.45
+#define SPECTRE_L2_FRACTION 0.9
 #endif
 // Two regions let one chunk's row pass run beside the previous chunk's slice
 // pass (measured on B200 for the bf16 long workload: 0.340 ms per mix with
