@@ -50,12 +50,14 @@ def test_shape_sweep_fp32(B, L, H, D, F):
 
 @pytest.mark.parametrize("B,L,H,D,F", [(1, 256, 1, 16, 40), (2, 12288, 2, 8, 6145),
                                        (1, 65536, 2, 8, 8192), (1, 3072, 3, 5, 1),
-                                       (1, 4096, 7, 72, 1000), (3, 4096, 4, 128, 2049)])
+                                       (1, 4096, 7, 72, 1000), (3, 4096, 4, 128, 2049),
+                                       (1, 65536, 7, 72, 8192)])
 def test_shape_sweep_bf16(B, L, H, D, F):
-    """bf16 shapes across the kernel variants: C = 504 (the last channel chunk
-    not a multiple of 64, so prefetching and plain row passes mix in one run;
-    dead lanes in the prefetching inverse pass) and C = 512 with B = 3 (the
-    persistent passes crossing batch boundaries)."""
+    """bf16 shapes across the kernel variants: C = 504 (dead lanes in the
+    prefetching inverse pass; at L = 65536 channel chunks of 128, 128, 128 and
+    120, the last not a multiple of 64, so the prefetching and the plain row
+    pass both run in one step, beside the tensor-core slice pass) and C = 512
+    with B = 3 (the persistent passes crossing batch boundaries)."""
     w = custom(B, L, H, D, F, dtype="bf16")
     inp = make_inputs(w)
     out, y = run_library(w, inp)
