@@ -78,6 +78,13 @@ enum spectre_status {
  *   F     : number of low-frequency rfft bins kept (F = L/2 + 1 keeps all).
  *   dtype : SPECTRE_F32 or SPECTRE_BF16.
  *   eps   : LayerNorm epsilon, > 0.
+ * Supported shapes: L = 2^k with 8 <= L <= 2^20, or L = 3 * 2^k with
+ * 12 <= L <= 786432 (else SPECTRE_ERR_UNSUPPORTED_L); B in [1, 65535],
+ * H, D >= 1 with C = H * D <= 2^20, 1 <= F <= L/2 + 1, and C narrow enough for
+ * the inverse pass to hold R token rows of all channels in shared memory:
+ * R * (C rounded up to a multiple of 32, plus 16) * 4 bytes <= 227 KiB, which
+ * is C <= 3616 for R = 16 (L <= 2^18, or L = 3 * 2^k <= 196608) and C <= 864
+ * for R = 64 (the longer L).  Other shapes give SPECTRE_ERR_ARG.
  */
 int spectre_mix_create(spectre_mix_t *out, int B, int L, int H, int D, int F,
                        int dtype, float eps);

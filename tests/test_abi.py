@@ -66,6 +66,10 @@ def test_error_strings_are_distinct():
     ((1, 1 << 21, 1, 16, 5, 0), "SPECTRE_ERR_UNSUPPORTED_L"),
     ((1, 5 * 1024, 1, 16, 5, 0), "SPECTRE_ERR_UNSUPPORTED_L"),
     ((1, 1 << 20, 8, 512, 5, 1), "SPECTRE_ERR_ARG"),     # C too wide for the R = 64 row pass
+    ((1, 1 << 20, 1, 865, 5, 1), "SPECTRE_ERR_ARG"),     # C = 865 > 864, the R = 64 limit
+    ((1, 1 << 18, 1, 3617, 5, 1), "SPECTRE_ERR_ARG"),    # C = 3617 > 3616, the R = 16 limit
+    ((65536, 256, 1, 16, 129, 0), "SPECTRE_ERR_ARG"),    # B above 65535
+    ((1, 256, 1024, 1025, 129, 0), "SPECTRE_ERR_ARG"),   # H * D above 2^20
 ])
 def test_create_validates_before_touching_the_device(args, code):
     from sub_quadratic_attention_b200 import binding as b

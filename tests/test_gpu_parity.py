@@ -271,3 +271,37 @@ def test_longest_slices_parked_product(case, dtype):
     out_ref, y_ref = oracle_full(w, inp)
     e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
     print(f"longest slices {w.name} {dtype}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+def test_widest_channels_r16():
+    """C = 3616, the widest plan with R = 16 (the inverse pass's shared-memory
+    variant holds 16 token rows of all channels: 227 KiB), against the oracle."""
+    w = custom(1, 4096, 4, 904, 2049, dtype="bf16")
+    inp = make_inputs(w)
+    out, y = run_library(w, inp)
+    out_ref, y_ref = oracle_full(w, inp)
+    e_out, e_y = check_parity(w, out, y, out_ref, y_ref)
+    print(f"widest R=16 {w.name}: rel-L2(out)={e_out:.3e} max|dy|={e_y:.3e}")
+
+
+def test_widest_channels_r64_zero_gate():
+    """C = 864, the widest plan with R = 64 (L = 2^19), checked by a property
+    that holds at any size: with G = 0 the mix is zero and y = LayerNorm(x).
+    Seeded inputs are drawn on the device (4 x 0.9 GB)."""
+    from sub_quadratic_attention_b200.binding import SpectreMix
+
+    B, L, H, D, F = 1, 2 ** 19, 1, 864, 5000
+    C = H * D
+    g = torch.Generator(device="cuda").manual_seed(864)
+    q, k, v, x = (torch.randn(B, L, C, generator=g, device="cuda").bfloat16() for _ in range(4))
+    G = torch.zeros(H, L // 2 + 1, device="cuda")
+    gamma = 1.0 + 0.1 * torch.randn(C, generator=g, device="cuda")
+    beta = 0.1 * torch.randn(C, generator=g, device="cuda")
+    with SpectreMix(B, L, H, D, F, "bf16") as mix:
+        assert mix.plan[0] == 64
+        y = mix(q, k, v, x, G, gamma, beta)
+        torch.cuda.synchronize()
+    ref = torch.nn.functional.layer_norm(x.float(), (C,), gamma, beta, eps=1e-5)
+    err = float((y.float() - ref).abs().max())
+    assert err <= 2e-2, err
+    print(f"widest R=64 zero gate: max|dy|={err:.3e}")
